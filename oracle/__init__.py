@@ -1,0 +1,112 @@
+"""FP64 CPU oracle for the scaled dot-product attention forward.
+
+TEST INFRASTRUCTURE ONLY.  The tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline / reference arm of ``bench.py`` may import this package; the
+product package (``scaled_dot_product_10_b200``) never does, and the oracle
+never imports the product.  The arithmetic lives in ``attn_oracle.c`` (plain
+C, FP64): it materialises S, masks it, takes the row max, exponentiates,
+normalises and multiplies by V, exactly as the definition
+``softmax(Q K^T / sqrt(d_k)) V`` on the rkmt.cn page (section 1) states.
+
+This module only marshals numpy arrays into that C function.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "attn_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lib = None
+
+
+def build(force: bool = False, src: str = _SRC, out: str = _LIB) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP, no fast-math: the FP64
+    arithmetic keeps IEEE semantics and program order)."""
+    if force or not os.path.exists(out) or os.path.getmtime(out) < os.path.getmtime(src):
+        cmd = ["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared",
+               "-fno-fast-math", "-ffp-contract=off", src, "-o", out, "-lm"]
+        subprocess.run(cmd, check=True)
+    return out
+
+
+def load(path: str | None = None):
+    """Load (building if needed) the oracle shared library."""
+    global _lib
+    if path is not None:
+        lib = ctypes.CDLL(path)
+    else:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+    lib.oracle_attn_fwd_f64.restype = ctypes.c_int
+    lib.oracle_attn_fwd_f64.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_double,
+        ctypes.c_void_p, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+    ]
+    lib.oracle_num_threads.restype = ctypes.c_int
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def num_threads() -> int:
+    return int(load().oracle_num_threads())
+
+
+def _as_bits(x) -> np.ndarray:
+    """Accept a torch bf16 tensor or a numpy uint16 array of bf16 bits."""
+    if isinstance(x, np.ndarray):
+        if x.dtype != np.uint16:
+            raise TypeError("numpy inputs must be uint16 arrays of bf16 bits")
+        return np.ascontiguousarray(x)
+    import torch  # local: only for the tensor -> bits view
+    if x.dtype != torch.bfloat16:
+        raise TypeError("torch inputs must be bfloat16")
+    return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
+
+
+def attn_fwd(q, k, v, causal: bool, scale: float, rows=None, want_p: bool = False, lib=None):
+    """Run the oracle.
+
+    q: [batch, s_q, h_q, d] bf16 (torch tensor or uint16 bits);
+    k, v: [batch, s_k, h_kv, d].
+    rows: None (every query row) or an int array [batch, h_q, n_rows] of the
+    query indices to evaluate per (batch, head).
+
+    Returns (o, lse, p): o [batch, h_q, n_rows, d] float64,
+    lse [batch, h_q, n_rows] float64 (natural log), p [batch, h_q, n_rows, s_k]
+    float64 or None.
+    """
+    qb, kb, vb = _as_bits(q), _as_bits(k), _as_bits(v)
+    batch, s_q, h_q, d = qb.shape
+    bk, s_k, h_kv, dk = kb.shape
+    if vb.shape != kb.shape or bk != batch or dk != d:
+        raise ValueError("shape mismatch between q, k and v")
+    if rows is None:
+        n_rows = s_q
+        rows_arr = None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+        if rows_arr.ndim != 3 or rows_arr.shape[:2] != (batch, h_q):
+            raise ValueError("rows must have shape [batch, h_q, n_rows]")
+        n_rows = rows_arr.shape[2]
+    o = np.zeros((batch, h_q, n_rows, d), dtype=np.float64)
+    lse = np.zeros((batch, h_q, n_rows), dtype=np.float64)
+    p = np.zeros((batch, h_q, n_rows, s_k), dtype=np.float64) if want_p else None
+    lib = lib or load()
+    rc = lib.oracle_attn_fwd_f64(
+        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
+        batch, h_q, h_kv, s_q, s_k, d, int(bool(causal)), float(scale),
+        None if rows_arr is None else rows_arr.ctypes.data, n_rows,
+        o.ctypes.data, lse.ctypes.data, None if p is None else p.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle rejected its arguments (code {rc})")
+    return o, lse, p

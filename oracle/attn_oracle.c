@@ -1,0 +1,187 @@
+/*
+ * attn_oracle.c -- plain FP64 CPU oracle for the scaled dot-product attention
+ * forward.  TEST INFRASTRUCTURE ONLY: the tests, the smoke check and the
+ * bench's CPU-baseline / reference arm may call it; the product path never
+ * does.  It shares no code, header, table or helper with the CUDA library.
+ *
+ * What it computes (the definition, written out with no blocking, fusion or
+ * reordering):
+ *
+ *   Attention(Q, K, V) = softmax(Q K^T / sqrt(d_k)) V
+ *       -- rkmt.cn "GPU attention operator optimisation" page, section 1
+ *          (the formula in the opening paragraph).
+ *
+ *   The three steps, in the order that page and the bjdmk.com.cn survey
+ *   page (section 1, "Query-Key product, softmax normalisation, Value
+ *   weighted sum") give them:
+ *     1. S[i][j] = scale * sum_c Q[i][c] * K[j][c]          (scores)
+ *        causal: S[i][j] = -inf for j > i                  (mask; the
+ *        intelliparadigm.com AVO page, section 2.2, fuses the mask into
+ *        the softmax -- here it is simply applied to S)
+ *     2. m_i = max_j S[i][j];  E = exp(S - m_i);  l_i = sum_j E[i][j];
+ *        P = E / l_i        (numerically stable softmax with the scale
+ *        applied before the max, as in the AVO page, section 3.1 item 2)
+ *     3. O[i][:] = sum_j P[i][j] V[j][:]
+ *   plus the per-row log-sum-exp of the scaled scores, LSE_i = m_i + ln l_i
+ *   (natural log; not on the pages -- the reading is stated in the design
+ *   notes).
+ *
+ *   Head sharing (grouped-query attention, rkmt.cn page section 3.2): query
+ *   head h reads key/value head h / (h_q / h_kv) -- contiguous groups.
+ *
+ * Layouts (all contiguous, row-major):
+ *   q   : bf16 bits [batch][s_q][h_q][d]
+ *   k,v : bf16 bits [batch][s_k][h_kv][d]
+ *   rows: int32 [batch][h_q][n_rows] query indices to evaluate (NULL: every
+ *         row 0..s_q-1, and n_rows must equal s_q)
+ *   o   : double [batch][h_q][n_rows][d]
+ *   lse : double [batch][h_q][n_rows]
+ *   p   : optional double [batch][h_q][n_rows][s_k] (the normalised P)
+ *
+ * BF16 inputs are decoded exactly (a bf16 value is the top half of an IEEE
+ * binary32), then widened to double; everything after that is FP64.
+ *
+ * Returns 0 on success, a negative code on a bad argument.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+static double bf16_bits_to_double(uint16_t bits)
+{
+    uint32_t u = ((uint32_t)bits) << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+/* Decode a whole bf16 array into doubles (done once so the inner loops read
+ * plain doubles). */
+static double *decode_bf16(const uint16_t *src, int64_t n)
+{
+    double *dst = (double *)malloc((size_t)n * sizeof(double));
+    if (!dst) return NULL;
+    for (int64_t i = 0; i < n; ++i) dst[i] = bf16_bits_to_double(src[i]);
+    return dst;
+}
+
+/* One (batch, query head) pair over a chunk of its requested rows.
+ * S is materialised for the chunk: n_chunk x s_k doubles. */
+static void attend_rows(const double *Q, const double *K, const double *V,
+                        int b, int h, int h_q, int h_kv, int s_q, int s_k,
+                        int d, int causal, double scale,
+                        const int32_t *rows, int r0, int r1, int n_rows,
+                        double *o, double *lse, double *p, double *S)
+{
+    const int group = h_q / h_kv;
+    const int g = h / group;                      /* key/value head */
+    const int64_t q_row_stride = (int64_t)h_q * d;  /* step of one token */
+    const int64_t kv_row_stride = (int64_t)h_kv * d;
+    const double *Qb = Q + (int64_t)b * s_q * q_row_stride + (int64_t)h * d;
+    const double *Kb = K + (int64_t)b * s_k * kv_row_stride + (int64_t)g * d;
+    const double *Vb = V + (int64_t)b * s_k * kv_row_stride + (int64_t)g * d;
+    const int64_t bh = (int64_t)b * h_q + h;
+
+    for (int r = r0; r < r1; ++r) {
+        const int i = rows ? rows[bh * n_rows + r] : r;
+        double *Srow = S + (int64_t)(r - r0) * s_k;
+
+        /* step 1: scores, then the causal mask */
+        for (int j = 0; j < s_k; ++j) {
+            double dot = 0.0;
+            for (int c = 0; c < d; ++c)
+                dot += Qb[(int64_t)i * q_row_stride + c] *
+                       Kb[(int64_t)j * kv_row_stride + c];
+            Srow[j] = scale * dot;
+            if (causal && j > i) Srow[j] = -INFINITY;
+        }
+
+        /* step 2: stable softmax over the row */
+        double m = -INFINITY;
+        for (int j = 0; j < s_k; ++j)
+            if (Srow[j] > m) m = Srow[j];
+        double l = 0.0;
+        for (int j = 0; j < s_k; ++j) {
+            Srow[j] = exp(Srow[j] - m); /* E[i][j]; exp(-inf) = 0 */
+            l += Srow[j];
+        }
+        for (int j = 0; j < s_k; ++j) Srow[j] = Srow[j] / l; /* P[i][j] */
+
+        if (p) memcpy(p + (bh * n_rows + r) * s_k, Srow, (size_t)s_k * sizeof(double));
+
+        /* step 3: P times V.  orow[c] accumulates P[j] * V[j][c] over
+         * j = 0, 1, ..., s_k-1 in that order (the loops are nested j-outer
+         * only so V is read row by row). */
+        double *orow = o + (bh * n_rows + r) * d;
+        for (int c = 0; c < d; ++c) orow[c] = 0.0;
+        for (int j = 0; j < s_k; ++j) {
+            const double *vrow = Vb + (int64_t)j * kv_row_stride;
+            for (int c = 0; c < d; ++c)
+                orow[c] += Srow[j] * vrow[c];
+        }
+        lse[bh * n_rows + r] = m + log(l);
+    }
+}
+
+int oracle_attn_fwd_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        int batch, int h_q, int h_kv, int s_q, int s_k, int d,
+                        int causal, double scale,
+                        const int32_t *rows, int n_rows,
+                        double *o, double *lse, double *p)
+{
+    if (!q || !k || !v || !o || !lse) return -1;
+    if (batch <= 0 || h_q <= 0 || h_kv <= 0 || s_q <= 0 || s_k <= 0 || d <= 0) return -2;
+    if (h_q % h_kv != 0) return -3;
+    if (n_rows <= 0 || (!rows && n_rows != s_q)) return -4;
+    if (rows) {
+        for (int64_t t = 0; t < (int64_t)batch * h_q * n_rows; ++t)
+            if (rows[t] < 0 || rows[t] >= s_q) return -5;
+    }
+    /* A causal row must see at least one key (row i sees keys 0..i). */
+    if (causal && s_q > s_k) return -6;
+
+    double *Q = decode_bf16(q, (int64_t)batch * s_q * h_q * d);
+    double *K = decode_bf16(k, (int64_t)batch * s_k * h_kv * d);
+    double *V = decode_bf16(v, (int64_t)batch * s_k * h_kv * d);
+    if (!Q || !K || !V) { free(Q); free(K); free(V); return -7; }
+
+    const int chunk = 32;
+    const int n_chunks = (n_rows + chunk - 1) / chunk;
+    const int64_t n_tasks = (int64_t)batch * h_q * n_chunks;
+    int failed = 0;
+
+#pragma omp parallel
+    {
+        double *S = (double *)malloc((size_t)chunk * s_k * sizeof(double));
+        if (!S) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < n_tasks; ++t) {
+            if (!S) continue;
+            const int64_t bh = t / n_chunks;
+            const int cidx = (int)(t % n_chunks);
+            const int b = (int)(bh / h_q), h = (int)(bh % h_q);
+            const int r0 = cidx * chunk;
+            const int r1 = r0 + chunk < n_rows ? r0 + chunk : n_rows;
+            attend_rows(Q, K, V, b, h, h_q, h_kv, s_q, s_k, d, causal, scale,
+                        rows, r0, r1, n_rows, o, lse, p, S);
+        }
+        free(S);
+    }
+    free(Q); free(K); free(V);
+    return failed ? -7 : 0;
+}
+
+/* Number of OpenMP threads the oracle will use (reported beside its timing). */
+int oracle_num_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

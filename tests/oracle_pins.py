@@ -1,0 +1,249 @@
+"""Pins that tie the FP64 oracle to facts fixed by the definition.
+
+Every pin takes the loaded oracle library (the real one, or a planted
+mutant in the mutation test) and raises AssertionError when the oracle
+disagrees with what the definition ``softmax(Q K^T * scale) V`` fixes
+(rkmt.cn page, section 1; the three steps of the bjdmk.com.cn page,
+section 1; the causal mask of the intelliparadigm.com AVO page,
+section 2.2; grouped heads, rkmt.cn page section 3.2).
+
+None of these re-types the oracle's formula: each compares against a
+closed form, an invariant of the definition, a hand derivation, or an
+independent library routine (torch's float64 SDPA on the CPU).
+"""
+from __future__ import annotations
+
+import glob
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+import oracle
+from scaled_dot_product_10_b200.workloads import make_qkv
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def bf16(a) -> torch.Tensor:
+    """Exact BF16 tensor from values that BF16 represents exactly."""
+    t = torch.as_tensor(np.asarray(a, dtype=np.float64)).to(torch.bfloat16)
+    back = t.to(torch.float64).numpy()
+    assert np.array_equal(back, np.asarray(a, dtype=np.float64)), "value not exact in bf16"
+    return t
+
+
+def f64(t: torch.Tensor) -> np.ndarray:
+    return t.to(torch.float64).numpy()
+
+
+def grid_values(rng, shape, lo=-2.0, hi=2.0, step=0.125):
+    """Random multiples of ``step`` in [lo, hi]: exact in BF16, and sums or
+    integer multiples of them stay exact."""
+    n = int(round((hi - lo) / step))
+    return lo + step * rng.integers(0, n + 1, size=shape)
+
+
+def run(lib, q, k, v, causal, scale, rows=None, want_p=False):
+    return oracle.attn_fwd(q, k, v, causal, scale, rows=rows, want_p=want_p, lib=lib)
+
+
+# ---------------------------------------------------------------------------
+
+
+def pin_rows_sum_to_one(lib):
+    """Softmax normalisation: each row of P sums to 1; masked entries are 0."""
+    q, k, v = make_qkv(1, 2, 2, 37, 37, seed=11, d=16)
+    for causal in (False, True):
+        _, _, p = run(lib, q, k, v, causal, 0.25, want_p=True)
+        assert np.all(np.abs(p.sum(-1) - 1.0) < 1e-12), "rows of P do not sum to 1"
+        assert np.all(p >= 0.0)
+        if causal:
+            i = np.arange(37)[:, None]
+            j = np.arange(37)[None, :]
+            assert np.all(p[..., j > i] == 0.0), "causal P is non-zero above the diagonal"
+            assert np.all(p[..., j <= i] > 0.0)
+
+
+def pin_identical_v_rows(lib):
+    """If every V row of a head equals v, the output of every query is v."""
+    rng = np.random.default_rng(5)
+    b, s, h_q, h_kv, d = 2, 19, 4, 2, 8
+    q, k, _ = make_qkv(b, h_q, h_kv, s, s, seed=12, d=d)
+    vrow = grid_values(rng, (b, 1, h_kv, d))
+    v = bf16(np.broadcast_to(vrow, (b, s, h_kv, d)).copy())
+    for causal in (False, True):
+        o, _, _ = run(lib, q, k, v, causal, 1 / math.sqrt(d))
+        for h in range(h_q):
+            g = h // (h_q // h_kv)
+            want = vrow[:, 0, g, :][:, None, :]
+            assert np.max(np.abs(o[:, h] - want)) < 1e-12, "identical V rows not reproduced"
+
+
+def pin_zero_query(lib):
+    """Q = 0 makes every visible score 0: O is the mean of the visible V rows
+    and LSE = ln(#visible keys) (s_k non-causal, i+1 causal)."""
+    b, s, h, d = 1, 29, 2, 8
+    _, k, v = make_qkv(b, h, h, s, s, seed=13, d=d)
+    q = torch.zeros((b, s, h, d), dtype=torch.bfloat16)
+    vv = f64(v)
+    o, lse, _ = run(lib, q, k, v, False, 0.3)
+    want = vv.mean(axis=1)  # [b, h, d]
+    assert np.max(np.abs(o - want[:, :, None, :])) < 1e-12, "Q=0: O is not the mean of V"
+    assert np.max(np.abs(lse - math.log(s))) < 1e-12, "Q=0: LSE is not ln(s_k)"
+    o, lse, _ = run(lib, q, k, v, True, 0.3)
+    for i in range(s):
+        want_i = vv[:, : i + 1].mean(axis=1)
+        assert np.max(np.abs(o[:, :, i] - want_i)) < 1e-12, "Q=0 causal: O is not the prefix mean"
+        assert np.max(np.abs(lse[:, :, i] - math.log(i + 1))) < 1e-12, "Q=0 causal: LSE != ln(i+1)"
+
+
+def pin_causal_row0(lib):
+    """Causal row 0 sees only key 0: O_0 = V_0 and LSE_0 = scale * q_0 . k_0."""
+    b, s, h, d = 2, 23, 3, 16
+    q, k, v = make_qkv(b, h, h, s, s, seed=14, d=d)
+    scale = 0.177
+    o, lse, _ = run(lib, q, k, v, True, scale)
+    qq, kk, vv = f64(q), f64(k), f64(v)
+    for bi in range(b):
+        for hi in range(h):
+            assert np.max(np.abs(o[bi, hi, 0] - vv[bi, 0, hi])) < 1e-12, "causal row 0 != V_0"
+            want = scale * float(np.dot(qq[bi, 0, hi], kk[bi, 0, hi]))
+            assert abs(lse[bi, hi, 0] - want) < 1e-12, "causal LSE_0 != scale q0.k0"
+
+
+def pin_key_shift(lib):
+    """Adding one vector c to every key row adds scale*q_i.c to every score of
+    row i: O is unchanged and LSE_i moves by scale*q_i.c (both modes)."""
+    rng = np.random.default_rng(6)
+    b, s, h, d = 1, 21, 2, 8
+    q = bf16(grid_values(rng, (b, s, h, d)))
+    kk = grid_values(rng, (b, s, h, d))
+    c = rng.integers(-2, 3, size=(b, 1, h, d)).astype(np.float64)
+    k0, k1 = bf16(kk), bf16(kk + c)
+    v = bf16(grid_values(rng, (b, s, h, d)))
+    scale = 0.25
+    qq = f64(q)
+    for causal in (False, True):
+        o0, l0, _ = run(lib, q, k0, v, causal, scale)
+        o1, l1, _ = run(lib, q, k1, v, causal, scale)
+        assert np.max(np.abs(o1 - o0)) < 1e-12, "key shift changed O"
+        shift = scale * np.einsum("bshd,bhd->bhs", qq, c[:, 0])
+        assert np.max(np.abs((l1 - l0) - shift)) < 1e-10, "key shift did not move LSE by scale*q.c"
+
+
+def pin_value_affine(lib):
+    """O is affine in V with weights summing to 1: V -> 2V + 1 gives O -> 2O + 1."""
+    rng = np.random.default_rng(7)
+    b, s, h, d = 1, 17, 2, 8
+    q, k, _ = make_qkv(b, h, h, s, s, seed=15, d=d)
+    vv = grid_values(rng, (b, s, h, d))
+    for causal in (False, True):
+        o0, l0, _ = run(lib, q, k, bf16(vv), causal, 0.4)
+        o1, l1, _ = run(lib, q, k, bf16(2 * vv + 1), causal, 0.4)
+        assert np.max(np.abs(o1 - (2 * o0 + 1))) < 1e-12, "O is not affine in V"
+        assert np.array_equal(l0, l1), "LSE depends on V"
+
+
+def pin_key_permutation(lib):
+    """Non-causal attention is a sum over keys: permuting the (K, V) rows
+    jointly changes neither O nor LSE."""
+    b, s, h, d = 2, 31, 2, 16
+    q, k, v = make_qkv(b, h, h, s, s, seed=16, d=d)
+    perm = torch.as_tensor(np.random.default_rng(8).permutation(s))
+    o0, l0, _ = run(lib, q, k, v, False, 0.25)
+    o1, l1, _ = run(lib, q, k[:, perm].contiguous(), v[:, perm].contiguous(), False, 0.25)
+    assert np.max(np.abs(o1 - o0)) < 1e-12 and np.max(np.abs(l1 - l0)) < 1e-12, \
+        "key permutation changed the result"
+
+
+def pin_gqa_equals_repeated_mha(lib):
+    """Grouped heads: h_q query heads over h_kv key/value heads equal plain
+    multi-head attention with each K/V head repeated h_q/h_kv times in a row."""
+    b, s, h_q, d = 2, 33, 8, 16
+    for h_kv in (2, 1):
+        q, k, v = make_qkv(b, h_q, h_kv, s, s, seed=17 + h_kv, d=d)
+        rep = h_q // h_kv
+        k_m = k.repeat_interleave(rep, dim=2).contiguous()
+        v_m = v.repeat_interleave(rep, dim=2).contiguous()
+        for causal in (False, True):
+            o0, l0, _ = run(lib, q, k, v, causal, 0.25)
+            o1, l1, _ = run(lib, q, k_m, v_m, causal, 0.25)
+            assert np.array_equal(o0, o1) and np.array_equal(l0, l1), "GQA != repeated MHA"
+
+
+def pin_torch_sdpa_f64(lib):
+    """Independent library routine: torch's float64 CPU scaled_dot_product_attention
+    (with is_causal and enable_gqa) gives the same O; the LSE matches
+    torch.logsumexp of the library matmul's scaled scores."""
+    cases = [(2, 4, 4, 67, 16), (1, 4, 2, 45, 128), (2, 8, 1, 40, 32)]
+    for b, h_q, h_kv, s, d in cases:
+        q, k, v = make_qkv(b, h_q, h_kv, s, s, seed=100 + s, d=d)
+        scale = 1 / math.sqrt(d)
+        qt = q.to(torch.float64).transpose(1, 2)
+        kt = k.to(torch.float64).transpose(1, 2)
+        vt = v.to(torch.float64).transpose(1, 2)
+        for causal in (False, True):
+            want = torch.nn.functional.scaled_dot_product_attention(
+                qt, kt, vt, is_causal=causal, scale=scale, enable_gqa=(h_q != h_kv))
+            o, lse, _ = run(lib, q, k, v, causal, scale)
+            assert np.max(np.abs(o - want.numpy())) < 1e-10, "O disagrees with torch SDPA (f64)"
+            kr = kt.repeat_interleave(h_q // h_kv, dim=1)
+            sc = torch.matmul(qt, kr.transpose(-1, -2)) * scale
+            if causal:
+                sc = sc.masked_fill(torch.ones(s, s, dtype=torch.bool).triu(1), float("-inf"))
+            want_lse = torch.logsumexp(sc, dim=-1).numpy()
+            assert np.max(np.abs(lse - want_lse)) < 1e-10, "LSE disagrees with torch.logsumexp"
+
+
+def _closed_form(expr: str) -> float:
+    return float(eval(expr, {"__builtins__": {}}, {"e": math.e, "log": math.log, "exp": math.exp}))
+
+
+def pin_golden_closed_forms(lib):
+    """Hand-derived tiny cases stored under tests/golden (each cites its passage)."""
+    files = sorted(glob.glob(os.path.join(GOLDEN, "*.json")))
+    assert files, "no golden fixtures"
+    for path in files:
+        with open(path) as f:
+            g = json.load(f)
+        q, k, v = bf16(g["q"]), bf16(g["k"]), bf16(g["v"])
+        o, lse, _ = run(lib, q, k, v, g["causal"], g["scale"])
+        want_o = np.vectorize(_closed_form)(np.array(g["expected_o"], dtype=object)).astype(np.float64)
+        want_l = np.vectorize(_closed_form)(np.array(g["expected_lse"], dtype=object)).astype(np.float64)
+        assert np.max(np.abs(o - want_o)) < 1e-14, f"{os.path.basename(path)}: O"
+        assert np.max(np.abs(lse - want_l)) < 1e-14, f"{os.path.basename(path)}: LSE"
+
+
+def pin_row_subset(lib):
+    """Evaluating a subset of rows gives those rows of the full evaluation."""
+    b, s, h, d = 1, 50, 2, 16
+    q, k, v = make_qkv(b, h, h, s, s, seed=21, d=d)
+    rows = np.array([[[0, 7, 31, 49], [3, 4, 5, 48]]], dtype=np.int32)
+    for causal in (False, True):
+        of, lf, _ = run(lib, q, k, v, causal, 0.2)
+        os_, ls, _ = run(lib, q, k, v, causal, 0.2, rows=rows)
+        for hi in range(h):
+            assert np.array_equal(os_[0, hi], of[0, hi, rows[0, hi]])
+            assert np.array_equal(ls[0, hi], lf[0, hi, rows[0, hi]])
+
+
+ALL_PINS = [
+    pin_rows_sum_to_one, pin_identical_v_rows, pin_zero_query, pin_causal_row0,
+    pin_key_shift, pin_value_affine, pin_key_permutation, pin_gqa_equals_repeated_mha,
+    pin_torch_sdpa_f64, pin_golden_closed_forms, pin_row_subset,
+]
+
+
+def failing_pins(lib) -> list[str]:
+    """Names of the pins the given oracle library fails (errors count as fails)."""
+    bad = []
+    for pin in ALL_PINS:
+        try:
+            with np.errstate(all="ignore"):
+                pin(lib)
+        except Exception as exc:  # noqa: BLE001 - any failure is a catch
+            bad.append(f"{pin.__name__}: {type(exc).__name__}")
+    return bad

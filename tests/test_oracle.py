@@ -1,0 +1,113 @@
+"""CPU tests of the FP64 oracle against its pins (no GPU needed)."""
+from __future__ import annotations
+
+import math
+import os
+import shutil
+import subprocess
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle_pins import ALL_PINS, failing_pins
+from scaled_dot_product_10_b200.workloads import make_qkv
+
+
+@pytest.fixture(scope="module")
+def lib():
+    return oracle.load()
+
+
+@pytest.mark.parametrize("pin", ALL_PINS, ids=lambda p: p.__name__)
+def test_oracle_pin(lib, pin):
+    pin(lib)
+
+
+def _brute_force(q, k, v, causal, scale):
+    """Per-element scalar evaluation in pure Python floats (tiny shapes only)."""
+    qq = q.float().double().tolist()
+    kk = k.float().double().tolist()
+    vv = v.float().double().tolist()
+    b, s_q, h_q, d = q.shape
+    _, s_k, h_kv, _ = k.shape
+    grp = h_q // h_kv
+    o = np.zeros((b, h_q, s_q, d))
+    lse = np.zeros((b, h_q, s_q))
+    for bi in range(b):
+        for h in range(h_q):
+            g = h // grp
+            for i in range(s_q):
+                scores = []
+                for j in range(s_k):
+                    if causal and j > i:
+                        continue
+                    acc = 0.0
+                    for c in range(d):
+                        acc += qq[bi][i][h][c] * kk[bi][j][g][c]
+                    scores.append((j, acc * scale))
+                mx = max(sv for _, sv in scores)
+                w = [(j, math.exp(sv - mx)) for j, sv in scores]
+                tot = sum(x for _, x in w)
+                for c in range(d):
+                    o[bi, h, i, c] = sum(x * vv[bi][j][g][c] for j, x in w) / tot
+                lse[bi, h, i] = mx + math.log(tot)
+    return o, lse
+
+
+@pytest.mark.parametrize("shape", [(1, 1, 1, 5, 4), (2, 4, 2, 17, 4), (1, 2, 1, 9, 128)])
+def test_oracle_brute_force(lib, shape):
+    b, h_q, h_kv, s, d = shape
+    q, k, v = make_qkv(b, h_q, h_kv, s, s, seed=31 + s, d=d)
+    for causal in (False, True):
+        o, lse, _ = oracle.attn_fwd(q, k, v, causal, 0.3, lib=lib)
+        ob, lb = _brute_force(q, k, v, causal, 0.3)
+        assert np.max(np.abs(o - ob)) < 1e-12
+        assert np.max(np.abs(lse - lb)) < 1e-12
+
+
+def test_oracle_rejects_bad_arguments(lib):
+    q, k, v = make_qkv(1, 4, 3, 8, 8, seed=1, d=4)   # 4 % 3 != 0
+    with pytest.raises(ValueError):
+        oracle.attn_fwd(q, k, v, False, 1.0, lib=lib)
+    q, k, v = make_qkv(1, 2, 2, 8, 4, seed=1, d=4)   # causal with s_q > s_k
+    with pytest.raises(ValueError):
+        oracle.attn_fwd(q, k, v, True, 1.0, lib=lib)
+
+
+# Planted mistakes: each is a plausible slip in the oracle's arithmetic.  A
+# mutant oracle is built from a copy of the source in a temporary directory
+# and must fail at least one pin.
+MUTANTS = {
+    "dropped_scale": ("Srow[j] = scale * dot;", "Srow[j] = dot;"),
+    "mask_wrong_side": ("if (causal && j > i)", "if (causal && j < i)"),
+    "mask_off_by_one": ("if (causal && j > i)", "if (causal && j > i + 1)"),
+    "gqa_modulo_mapping": ("const int g = h / group;", "const int g = h % h_kv;"),
+    "transposed_scores": ("dot += Qb[(int64_t)i * q_row_stride + c] *\n                       Kb[(int64_t)j * kv_row_stride + c];",
+                          "dot += Qb[(int64_t)j * q_row_stride + c] *\n                       Kb[(int64_t)i * kv_row_stride + c];"),
+    "dropped_first_term": ("for (int c = 0; c < d; ++c)\n                dot +=", "for (int c = 1; c < d; ++c)\n                dot +="),
+    "no_max_subtraction": ("Srow[j] = exp(Srow[j] - m);", "Srow[j] = exp(Srow[j]);"),
+    "exp_sign_flip": ("Srow[j] = exp(Srow[j] - m);", "Srow[j] = exp(m - Srow[j]);"),
+    "min_instead_of_max": ("if (Srow[j] > m) m = Srow[j];", "if (Srow[j] < m) m = Srow[j];"),
+    "no_normalisation": ("Srow[j] = Srow[j] / l;", "Srow[j] = Srow[j];"),
+    "lse_missing_max": ("m + log(l);", "log(l);"),
+    "lse_log2": ("m + log(l);", "m + log2(l);"),
+    "k_used_as_v": ("const double *vrow = Vb +", "const double *vrow = Kb +"),
+    "mask_to_zero": ("Srow[j] = -INFINITY;", "Srow[j] = 0.0;"),
+    "bf16_decode_shift": ("((uint32_t)bits) << 16", "((uint32_t)bits) << 15"),
+}
+
+
+@pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_planted_mistake_is_caught(tmp_path, name):
+    src = open(os.path.join(os.path.dirname(oracle.__file__), "attn_oracle.c")).read()
+    old, new = MUTANTS[name]
+    assert src.count(old) >= 1, f"mutation site for {name} not found"
+    mut = tmp_path / "mutant.c"
+    mut.write_text(src.replace(old, new, 1))
+    so = tmp_path / "mutant.so"
+    subprocess.run(["gcc", "-O2", "-std=c11", "-fopenmp", "-fPIC", "-shared", str(mut), "-o", str(so), "-lm"],
+                   check=True)
+    bad = failing_pins(oracle.load(str(so)))
+    assert bad, f"planted mistake '{name}' passed every pin"
