@@ -1,0 +1,411 @@
+#!/usr/bin/env python
+"""Throughput of the fused attention forward on B200.
+
+One step = the whole hot path over one batch: a non-causal and a causal
+forward of the MHA workload (batch 8, 16 heads, sequence 4096, head dim 128,
+BF16), inputs resident in HBM.  The metric is attention-forward TFLOPS,
+counting 4*b*h*s_q*s_k*d FLOPs per forward, halved for the causal one.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) are replicas: each
+rank runs its own batch (weak scaling), timed on the device, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from scaled_dot_product_10_b200.workloads import WORKLOADS, sample_rows, workload_qkv  # noqa: E402
+
+METRIC = "attn fwd TFLOPS (bf16, d=128, causal & non-causal) and % of B200 BF16 peak"
+UNIT = "TFLOPS"
+SPEC_PEAK_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0}
+MODES = (False, True)  # non-causal, causal
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=400)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default="mha_b8_h16_s4096", choices=sorted(WORKLOADS))
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(glob.glob(os.path.join(ROOT, "scaled_dot_product_10_b200", "csrc", "*"))):
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken
+    on the current kernel sources; else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        d = json.load(f)
+    if d.get("kernel_hash") != kernel_source_hash() or d.get("workload") != workload:
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML (read-only) while
+    the timed region runs."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index: int, period_s: float = 0.02):
+        self.samples, self.reasons, self.max_mhz = [], set(), None
+        self._stop = threading.Event()
+        self._period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nv = pynvml
+            uuid = None
+            try:
+                uuid = torch.cuda.get_device_properties(index).uuid
+            except Exception:
+                pass
+            self._h = None
+            if uuid is not None:
+                for i in range(pynvml.nvmlDeviceGetCount()):
+                    h = pynvml.nvmlDeviceGetHandleByIndex(i)
+                    u = pynvml.nvmlDeviceGetUUID(h)
+                    u = u.decode() if isinstance(u, bytes) else u
+                    if str(uuid) in u:
+                        self._h = h
+            if self._h is None:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self._nv = None
+
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def __enter__(self):
+        if self._nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        if self._nv is not None:
+            self._stop.set()
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ------------------------------------------------------------------ oracle arm
+def oracle_sample_rate(w, target_s: float, seed_offset: int = 0):
+    """Time the FP64 oracle on a bounded row sample of the workload (both
+    masks).  Returns (TFLOPS in the metric's convention, seconds, rows/head,
+    threads)."""
+    import oracle
+    q, k, v = workload_qkv(w)
+    d = 128
+
+    def flops(rows, causal):
+        if causal:
+            return float(4 * d * (rows.astype("int64") + 1).sum())
+        return float(4 * d * w.seq * rows.size)
+
+    def run(n_rows, seed):
+        rows = sample_rows(w.batch, w.h_q, w.seq, n_rows, seed=seed)
+        t0 = time.perf_counter()
+        f = 0.0
+        for causal in MODES:
+            oracle.attn_fwd(q, k, v, causal, w.scale, rows=rows)
+            f += flops(rows, causal)
+        return f, time.perf_counter() - t0
+
+    f1, t1 = run(1, w.seed + 1 + seed_offset)            # calibration
+    per_row = t1 / max(1, w.batch * w.h_q)
+    n = max(1, min(w.seq, int(target_s / max(per_row * w.batch * w.h_q, 1e-9))))
+    f, t = run(n, w.seed + 2 + seed_offset)
+    return f / t / 1e12, t, n, oracle.num_threads()
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return 0
+    w = WORKLOADS[args.workload]
+    budget = 150.0
+    per_step = budget / max(1, args.steps + args.warmup)
+    import oracle
+    q, k, v = workload_qkv(w)
+    d = 128
+    times, flops_total = [], 0.0
+    rows_n = None
+    for i in range(args.warmup + args.steps):
+        if rows_n is None:
+            rows_n = 1
+        rows = sample_rows(w.batch, w.h_q, w.seq, rows_n, seed=w.seed + 100 + i)
+        t0 = time.perf_counter()
+        f = 0.0
+        for causal in MODES:
+            oracle.attn_fwd(q, k, v, causal, w.scale, rows=rows)
+            f += float(4 * d * ((rows.astype("int64") + 1).sum() if causal else w.seq * rows.size))
+        dt = time.perf_counter() - t0
+        if i < args.warmup:
+            # size the sample so one step costs about `per_step` seconds
+            rows_n = max(1, min(w.seq, int(rows_n * per_step / max(dt, 1e-6))))
+            continue
+        times.append(dt)
+        flops_total += f
+    total_t = sum(times)
+    value = flops_total / total_t / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_t / len(times),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv,
+                   "seq": w.seq, "head_dim": 128, "modes": ["noncausal", "causal"]},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"{rows_n} seeded query rows per (batch, head) per step, both masks"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, world, rank, local):
+    from scaled_dot_product_10_b200 import attn
+
+    w = WORKLOADS[args.workload]
+    attn.load_library()
+    q, k, v = workload_qkv(w)
+    if rank:
+        # replicas: each rank runs its own batch of the same shape
+        g = torch.Generator().manual_seed(w.seed + rank)
+        q = torch.randn(q.shape, generator=g).to(torch.bfloat16)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    od = torch.empty_like(qd)
+    ld = torch.empty((w.batch, w.h_q, w.seq), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    qp, kp, vp, op, lp = qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), od.data_ptr(), ld.data_ptr()
+
+    def launch(causal):
+        rc = attn.attn_fwd_raw(qp, kp, vp, op, lp, w.batch, w.h_q, w.h_kv, w.seq, w.seq, 128,
+                               causal, w.scale, sh)
+        if rc != attn.ATTN_OK:
+            raise attn.AttnError(rc, "attn_fwd")
+
+    for _ in range(args.warmup):
+        for causal in MODES:
+            launch(causal)
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = {m: [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(K)] for m in MODES}
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    with sampler:
+        t_start.record(stream)
+        for i in range(K):
+            for causal in MODES:
+                a, b = ev[causal][i]
+                a.record(stream)
+                launch(causal)
+                b.record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    barrier(world)
+    rc = attn.attn_status()
+    if rc != attn.ATTN_OK:
+        raise attn.AttnError(rc, "kernel status after the timed region")
+
+    total_ms = max_over_ranks(t_start.elapsed_time(t_end), world)
+    launch_ms = {m: sum(a.elapsed_time(b) for a, b in ev[m]) / K for m in MODES}
+    flops_step = sum(w.flops(m) for m in MODES)
+    value = world * flops_step * K / (total_ms * 1e-3) / 1e12
+
+    peaks, peak_src = load_peaks()
+    achieved = flops_step / (sum(launch_ms.values()) * 1e-3) / 1e12
+    peak = float(peaks["bf16_tflops"])
+    traffic = committed_traffic(w.name)
+    roofline = {
+        "bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        "frac": achieved / peak,
+        "traffic": (sum(traffic[m] for m in ("noncausal", "causal")) / 2 if traffic else None),
+        "peak_source": f"{peak_src} bf16 burst (cuBLAS 8192^3)",
+        "frac_of_sustained": achieved / float(peaks.get("bf16_tflops_sustained", peak)),
+        "frac_of_spec_2250": achieved / SPEC_PEAK_TFLOPS,
+        "kernel": "attn_fwd_sm100_kernel",
+    }
+    modes = {("causal" if m else "noncausal"): {
+        "ms_per_launch": launch_ms[m], "tflops": w.flops(m) / (launch_ms[m] * 1e-3) / 1e12}
+        for m in MODES}
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) BF16; inputs 402 MB > 126 MB L2, no flush needed)",
+        "config": {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv,
+                   "seq": w.seq, "head_dim": 128, "modes": ["noncausal", "causal"],
+                   "l2": "inputs larger than L2", "parallelism": f"replicas x{world}"},
+        "modes": modes,
+        "pct_of_spec_peak": 100.0 * value / world / SPEC_PEAK_TFLOPS,
+        "roofline": roofline,
+        "clocks": sampler.summary(),
+        "gpu_launches": 2 * K,
+        "kernel_hash": kernel_source_hash(),
+    }
+
+    if not args.no_e2e:
+        line["e2e"] = run_e2e(args, w, q, k, v, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tfl, secs, n, cores = oracle_sample_rate(w, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": tfl, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{n} seeded query rows per (batch, head) of {w.name}, both masks, "
+                      f"{secs:.1f} s; FLOPs counted as 4*d*visible keys per row"}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, q, k, v, world):
+    """Same metric through the host-buffer C entry point: pinned host inputs,
+    H2D copies, the forward, and D2H of O and LSE inside the timed region."""
+    from scaled_dot_product_10_b200 import attn
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((w.batch, w.h_q, w.seq), dtype=torch.float32).pin_memory()
+    ws = torch.empty(attn.host_workspace_bytes(w.batch, w.h_q, w.h_kv, w.seq, w.seq),
+                     dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for causal in MODES:
+            attn.attn_fwd_host(qh, kh, vh, oh, lh, ws, causal=causal, scale=w.scale,
+                               stream=stream)
+
+    step()
+    torch.cuda.synchronize()
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    a.record(stream)
+    for _ in range(args.e2e_steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(b), world)
+    flops_step = sum(w.flops(m) for m in MODES)
+    n_in = sum(t.numel() * t.element_size() for t in (qh, kh, vh))
+    n_out = oh.numel() * oh.element_size() + lh.numel() * lh.element_size()
+    return {"value": world * flops_step * args.e2e_steps / (ms * 1e-3) / 1e12, "unit": UNIT,
+            "h2d_bytes_per_step": len(MODES) * n_in, "d2h_bytes_per_step": len(MODES) * n_out,
+            "steps": args.e2e_steps, "ms_per_step": ms / args.e2e_steps}
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        return run_reference(args, world, rank)
+    world, rank, local = dist_setup(args)
+    try:
+        run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,127 @@
+/*
+ * attn_fwd.h -- C ABI of the B200 (sm_100a) fused scaled dot-product
+ * attention forward.
+ *
+ * The operation (rkmt.cn "GPU attention operator optimisation" page,
+ * section 1; the three steps of the bjdmk.com.cn survey page, section 1):
+ *
+ *     S   = scale * Q K^T                  (per batch and query head)
+ *     S   = S with S[i][j] = -inf for j > i          (causal mode only; the
+ *           mask of the intelliparadigm.com AVO page, section 2.2)
+ *     O   = softmax_rows(S) V
+ *     LSE = log(sum_j exp(S[i][j]))        (natural log, per query row)
+ *
+ * Grouped-query / multi-query attention (rkmt.cn page, section 3.2): query
+ * head h reads key/value head h / (h_q / h_kv); h_kv == h_q is plain
+ * multi-head attention, h_kv == 1 is multi-query attention.
+ *
+ * Numerics: Q, K, V are BF16; Q K^T and P V accumulate in FP32 on the tensor
+ * cores; the softmax runs in FP32 (the precision split of the bjdmk.com.cn
+ * page, section 3); the probabilities P are rounded to BF16 before the P V
+ * product; O is written as BF16 (round to nearest even), LSE as FP32.
+ * NaN or Inf in the inputs propagate; they are not checked.
+ *
+ * Every function returns an attn_status_t code.  On any error nothing is
+ * written to o or lse.
+ */
+#ifndef SDPA10_ATTN_FWD_H
+#define SDPA10_ATTN_FWD_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    ATTN_OK = 0,
+    ATTN_ERR_INVALID = 1,     /* null pointer, dimension <= 0, h_q % h_kv != 0,
+                                 non-finite scale, size beyond the kernel's
+                                 32-bit tile indexing, workspace too small */
+    ATTN_ERR_UNSUPPORTED = 2, /* d != 128, or causal with s_q != s_k */
+    ATTN_ERR_ALIGN = 3,       /* a q/k/v/o pointer not 16-byte aligned (TMA),
+                                 or lse not 4-byte aligned */
+    ATTN_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (no device,
+                                 launch failure, ...) */
+    ATTN_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (reported by
+                                 attn_status) */
+} attn_status_t;
+
+/*
+ * attn_fwd -- launch the fused forward on `stream` (a cudaStream_t; NULL is
+ * the legacy default stream) and return without synchronising.
+ *
+ *   q    device, bf16 [batch, s_q, h_q,  d] contiguous (read)
+ *   k    device, bf16 [batch, s_k, h_kv, d] contiguous (read)
+ *   v    device, bf16 [batch, s_k, h_kv, d] contiguous (read)
+ *   o    device, bf16 [batch, s_q, h_q,  d] contiguous (written)
+ *   lse  device, fp32 [batch, h_q, s_q]     contiguous (written)
+ *   d     must be 128
+ *   causal  0: full attention; 1: key j is visible to query i iff j <= i
+ *           (requires s_q == s_k)
+ *   scale   multiplies Q K^T before the softmax (usually 1/sqrt(d))
+ *
+ * The caller owns every buffer; the call allocates nothing.  o and lse must
+ * not overlap the inputs.  q/k/v/o must be 16-byte aligned, lse 4-byte
+ * aligned.  The kernel's device-side waits are bounded: if one gives up, the
+ * kernel exits early (o/lse then hold unspecified values) and the next
+ * attn_status call reports ATTN_ERR_TIMEOUT.
+ */
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int batch, int h_q, int h_kv, int s_q, int s_k, int d,
+             int causal, float scale, void* stream);
+
+/*
+ * attn_fwd_host -- the same forward on HOST buffers: copies q, k, v to the
+ * device (cudaMemcpyAsync on `stream`), runs attn_fwd, copies o and lse back,
+ * and returns without synchronising (the caller synchronises `stream` before
+ * reading o/lse; pinned host memory makes the copies asynchronous).
+ *
+ *   q, k, v, o, lse   host pointers with the layouts of attn_fwd
+ *   workspace         device buffer of at least
+ *                     attn_fwd_host_workspace_bytes(...) bytes, 256-byte
+ *                     aligned, owned by the caller
+ */
+int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                  int batch, int h_q, int h_kv, int s_q, int s_k, int d,
+                  int causal, float scale, void* workspace, size_t workspace_bytes,
+                  void* stream);
+
+/* Device workspace bytes attn_fwd_host needs for these sizes (0 on bad sizes). */
+size_t attn_fwd_host_workspace_bytes(int batch, int h_q, int h_kv, int s_q, int s_k, int d);
+
+/*
+ * attn_status -- synchronise `stream`, then read and clear the calling
+ * device's kernel status word.  Returns ATTN_OK, ATTN_ERR_TIMEOUT if a kernel
+ * launched since the last call gave up a bounded wait, or ATTN_ERR_CUDA if
+ * the synchronisation itself failed.
+ */
+int attn_status(void* stream);
+
+/* Static, human-readable text for a status code. */
+const char* attn_strerror(int code);
+
+/*
+ * attn_set_wait_timeout_ns -- bound (nanoseconds) on every device-side wait
+ * of kernels launched afterwards by this process (default 2e9 = 2 s;
+ * 0 restores the default).
+ */
+int attn_set_wait_timeout_ns(uint64_t ns);
+
+/*
+ * attn_selftest_wait_timeout -- launch one CTA that waits on a barrier
+ * nothing ever arrives on, bounded by `timeout_ns`; the wait gives up, the
+ * kernel sets the status word and exits.  A following attn_status returns
+ * ATTN_ERR_TIMEOUT.  Exercises the bounded-wait path without faulting.
+ */
+int attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
+
+/* Number of kernel launches the last attn_fwd / attn_fwd_host made (1). */
+int attn_last_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SDPA10_ATTN_FWD_H */

@@ -1,0 +1,167 @@
+"""ctypes binding of the C ABI in ``include/attn_fwd.h``.
+
+Argument marshalling only: every step of the forward runs in the CUDA
+library.  Loading fails loudly if the library is missing -- there is no
+fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+ATTN_OK = 0
+ATTN_ERR_INVALID = 1
+ATTN_ERR_UNSUPPORTED = 2
+ATTN_ERR_ALIGN = 3
+ATTN_ERR_CUDA = 4
+ATTN_ERR_TIMEOUT = 5
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_NAME = "libattn_sm100.so"
+_lib = None
+
+# (name, restype, argtypes) of every exported entry point.
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_SIGNATURES = [
+    ("attn_fwd", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]),
+    ("attn_fwd_host", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
+                           _P, ctypes.c_size_t, _P]),
+    ("attn_fwd_host_workspace_bytes", ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
+    ("attn_status", _I, [_P]),
+    ("attn_strerror", ctypes.c_char_p, [_I]),
+    ("attn_set_wait_timeout_ns", _I, [ctypes.c_uint64]),
+    ("attn_selftest_wait_timeout", _I, [ctypes.c_uint64, _P]),
+    ("attn_last_launch_count", _I, []),
+]
+EXPORTED = [s[0] for s in _SIGNATURES]
+
+
+class AttnError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {attn_strerror(code)} (code {code})")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, _LIB_NAME)
+
+
+def load_library(path: str | None = None):
+    """Load the CUDA library (raises OSError if it is not built)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or library_path()
+    if not os.path.exists(p):
+        raise OSError(f"{p} is missing: build it with `python -m scaled_dot_product_10_b200.build`")
+    lib = ctypes.CDLL(p)
+    for name, res, args in _SIGNATURES:
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def attn_strerror(code: int) -> str:
+    return load_library().attn_strerror(int(code)).decode()
+
+
+def _stream_handle(stream) -> int | None:
+    if stream is None:
+        import torch
+        return torch.cuda.current_stream().cuda_stream
+    if isinstance(stream, int):
+        return stream
+    return stream.cuda_stream
+
+
+def _check_qkv(q, k, v):
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16:
+            raise TypeError(f"{name} must be bfloat16")
+        if t.dim() != 4:
+            raise ValueError(f"{name} must be [batch, seq, heads, head_dim]")
+        if not t.is_contiguous():
+            raise ValueError(f"{name} must be contiguous")
+    b, s_q, h_q, d = q.shape
+    bk, s_k, h_kv, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or bk != b or dk != d:
+        raise ValueError("q, k, v shapes disagree")
+    return b, s_q, h_q, h_kv, s_k, d
+
+
+def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, lse=None,
+             stream=None):
+    """O, LSE = attention forward on CUDA tensors [batch, seq, heads, 128] (BF16).
+
+    Returns (o [b, s_q, h_q, 128] BF16, lse [b, h_q, s_q] FP32).  Asynchronous
+    on ``stream`` (default: torch's current stream).
+    """
+    import torch
+    b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
+    rc = load_library().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                 lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d, int(bool(causal)),
+                                 float(scale), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd")
+    return o, lse
+
+
+def attn_fwd_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, b, h_q, h_kv, s_q, s_k, d, causal, scale,
+                 stream_handle) -> int:
+    """Direct call of the C entry point; returns its status code."""
+    return load_library().attn_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, b, h_q, h_kv, s_q, s_k,
+                                   d, int(causal), float(scale), stream_handle)
+
+
+def host_workspace_bytes(b, h_q, h_kv, s_q, s_k, d=128) -> int:
+    return int(load_library().attn_fwd_host_workspace_bytes(b, h_q, h_kv, s_q, s_k, d))
+
+
+def attn_fwd_host(q, k, v, o, lse, workspace, causal: bool = False, scale: float | None = None,
+                  stream=None):
+    """Forward on HOST tensors (pinned for asynchronous copies) through the
+    C entry point that copies in, runs and copies out.  ``workspace`` is a
+    CUDA uint8 tensor of at least :func:`host_workspace_bytes` bytes."""
+    b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    rc = load_library().attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
+                                      int(bool(causal)), float(scale), workspace.data_ptr(),
+                                      workspace.numel() * workspace.element_size(),
+                                      _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_host")
+    return o, lse
+
+
+def attn_status(stream=None) -> int:
+    """Synchronise the stream, then read and clear the device status word."""
+    return int(load_library().attn_status(_stream_handle(stream)))
+
+
+def set_wait_timeout_ns(ns: int) -> None:
+    load_library().attn_set_wait_timeout_ns(int(ns))
+
+
+def selftest_wait_timeout(timeout_ns: int, stream=None) -> int:
+    return int(load_library().attn_selftest_wait_timeout(int(timeout_ns), _stream_handle(stream)))
+
+
+def last_launch_count() -> int:
+    return int(load_library().attn_last_launch_count())

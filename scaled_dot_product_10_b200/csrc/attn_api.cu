@@ -1,0 +1,251 @@
+// attn_api.cu -- the C ABI declared in include/attn_fwd.h: argument
+// validation (no CUDA call on an invalid argument), TMA descriptor encoding,
+// the persistent launch, and the per-device status word.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <mutex>
+
+#include "attn_fwd.h"
+#include "attn_fwd_kernel.cuh"
+
+namespace {
+
+using namespace sdpa10;
+
+constexpr int kKvStages = 4;
+using Layout = SmemLayout<kKvStages>;
+constexpr int kThreads = 192;
+constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
+// Bytes of K/V that the tiles running at one time should share through L2.
+constexpr size_t kL2SectionBytes = 48ull << 20;
+constexpr int kMaxDevices = 64;
+
+// Per-device status word: bit 0 = a bounded wait gave up.
+__device__ unsigned int g_status_word;
+
+struct DeviceState {
+    bool ready = false;
+    int num_sms = 0;
+    unsigned int* status = nullptr;  // device address of g_status_word
+};
+
+std::mutex g_mutex;
+DeviceState g_dev[kMaxDevices];
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+unsigned long long g_timeout_ns = kDefaultTimeoutNs;
+int g_last_launches = 0;
+
+int init_device(int dev, DeviceState** out) {
+    if (dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_mutex);
+    DeviceState& st = g_dev[dev];
+    if (!st.ready) {
+        if (!g_encode) {
+            void* fn = nullptr;
+            cudaDriverEntryPointQueryResult q;
+            if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+                    cudaSuccess ||
+                q != cudaDriverEntryPointSuccess || fn == nullptr)
+                return ATTN_ERR_CUDA;
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+        }
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        if (cudaFuncSetAttribute(attn_fwd_sm100_kernel<kKvStages>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Layout::kAlloc) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        void* sp = nullptr;
+        if (cudaGetSymbolAddress(&sp, g_status_word) != cudaSuccess) return ATTN_ERR_CUDA;
+        st.num_sms = sms;
+        st.status = static_cast<unsigned int*>(sp);
+        st.ready = true;
+    }
+    *out = &st;
+    return ATTN_OK;
+}
+
+// [batch, seq, heads, 128] BF16 as a 4-D tensor map {d, heads, seq, batch},
+// box {64, 1, 128, 1} (one 128-byte swizzled half of a 128-row tile).
+bool encode_map(CUtensorMap* m, const void* base, int heads, int seq, int batch) {
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(heads),
+                          static_cast<cuuint64_t>(seq), static_cast<cuuint64_t>(batch)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHeadDim) * 2,
+                             static_cast<cuuint64_t>(heads) * kHeadDim * 2,
+                             static_cast<cuuint64_t>(seq) * heads * kHeadDim * 2};
+    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int validate_sizes(int batch, int h_q, int h_kv, int s_q, int s_k, int d) {
+    if (batch <= 0 || h_q <= 0 || h_kv <= 0 || s_q <= 0 || s_k <= 0 || d <= 0)
+        return ATTN_ERR_INVALID;
+    if (h_q % h_kv != 0) return ATTN_ERR_INVALID;
+    if (d != kHeadDim) return ATTN_ERR_UNSUPPORTED;
+    const long long n_qb = (s_q + kBlockM - 1) / kBlockM;
+    if (static_cast<long long>(batch) * h_q * n_qb > 0x7fffffffLL) return ATTN_ERR_INVALID;
+    return ATTN_OK;
+}
+
+int validate(const void* q, const void* k, const void* v, const void* o, const float* lse,
+             int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal, float scale) {
+    if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
+    int rc = validate_sizes(batch, h_q, h_kv, s_q, s_k, d);
+    if (rc != ATTN_OK) return rc;
+    if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
+    if (!(scale > 0.f)) return ATTN_ERR_UNSUPPORTED;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID;
+    if (causal && s_q != s_k) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+        !aligned(lse, 4))
+        return ATTN_ERR_ALIGN;
+    return ATTN_OK;
+}
+
+size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+}  // namespace
+
+extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal,
+                        float scale, void* stream) {
+    int rc = validate(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale);
+    if (rc != ATTN_OK) return rc;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    DeviceState* st = nullptr;
+    rc = init_device(dev, &st);
+    if (rc != ATTN_OK) return rc;
+
+    CUtensorMap tq, tk, tv;
+    if (!encode_map(&tq, q, h_q, s_q, batch) || !encode_map(&tk, k, h_kv, s_k, batch) ||
+        !encode_map(&tv, v, h_kv, s_k, batch))
+        return ATTN_ERR_CUDA;
+
+    FwdParams p{};
+    p.batch = batch;
+    p.h_q = h_q;
+    p.h_kv = h_kv;
+    p.s_q = s_q;
+    p.s_k = s_k;
+    p.group = h_q / h_kv;
+    p.n_qb = (s_q + kBlockM - 1) / kBlockM;
+    p.n_kb = (s_k + kBlockN - 1) / kBlockN;
+    p.causal = causal;
+    p.num_tiles = batch * h_q * p.n_qb;
+    const size_t unit_bytes = 2ull * s_k * kHeadDim * 2;  // K and V of one (batch, kv head)
+    const size_t per_sec = kL2SectionBytes / (unit_bytes ? unit_bytes : 1);
+    const int units_total = batch * h_kv;
+    p.units_per_section = static_cast<int>(per_sec < 1 ? 1 : (per_sec > (size_t)units_total ? units_total : per_sec));
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    p.timeout_ns = g_timeout_ns;
+    p.status = st->status;
+
+    const int grid = p.num_tiles < st->num_sms ? p.num_tiles : st->num_sms;
+    attn_fwd_sm100_kernel<kKvStages><<<grid, kThreads, Layout::kAlloc,
+                                       static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, p);
+    g_last_launches = 1;
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
+extern "C" size_t attn_fwd_host_workspace_bytes(int batch, int h_q, int h_kv, int s_q, int s_k,
+                                                int d) {
+    if (validate_sizes(batch, h_q, h_kv, s_q, s_k, d) != ATTN_OK) return 0;
+    const size_t qb = static_cast<size_t>(batch) * s_q * h_q * d * 2;
+    const size_t kb = static_cast<size_t>(batch) * s_k * h_kv * d * 2;
+    const size_t lb = static_cast<size_t>(batch) * h_q * s_q * 4;
+    return round_up(qb, 256) * 2 + round_up(kb, 256) * 2 + round_up(lb, 256);
+}
+
+extern "C" int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal,
+                             float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    int rc = validate(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale);
+    if (rc != ATTN_OK) return rc;
+    if (!workspace) return ATTN_ERR_INVALID;
+    if (!aligned(workspace, 256)) return ATTN_ERR_ALIGN;
+    const size_t need = attn_fwd_host_workspace_bytes(batch, h_q, h_kv, s_q, s_k, d);
+    if (workspace_bytes < need) return ATTN_ERR_INVALID;
+    const size_t qb = static_cast<size_t>(batch) * s_q * h_q * d * 2;
+    const size_t kb = static_cast<size_t>(batch) * s_k * h_kv * d * 2;
+    const size_t lb = static_cast<size_t>(batch) * h_q * s_q * 4;
+    char* w = static_cast<char*>(workspace);
+    char* dq = w;
+    char* dk = dq + round_up(qb, 256);
+    char* dv = dk + round_up(kb, 256);
+    char* d_o = dv + round_up(kb, 256);
+    float* dl = reinterpret_cast<float*>(d_o + round_up(qb, 256));
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(dq, q, qb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dk, k, kb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
+        cudaMemcpyAsync(dv, v, kb, cudaMemcpyHostToDevice, s) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    rc = attn_fwd(dq, dk, dv, d_o, dl, batch, h_q, h_kv, s_q, s_k, d, causal, scale, stream);
+    if (rc != ATTN_OK) return rc;
+    if (cudaMemcpyAsync(o, d_o, qb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+        cudaMemcpyAsync(lse, dl, lb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
+extern "C" int attn_status(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    unsigned int word = 0;
+    if (cudaMemcpyFromSymbol(&word, g_status_word, sizeof(word)) != cudaSuccess)
+        return ATTN_ERR_CUDA;
+    if (word != 0) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(g_status_word, &zero, sizeof(zero)) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        return ATTN_ERR_TIMEOUT;
+    }
+    return ATTN_OK;
+}
+
+extern "C" const char* attn_strerror(int code) {
+    switch (code) {
+        case ATTN_OK: return "success";
+        case ATTN_ERR_INVALID: return "invalid argument";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (d must be 128; causal needs s_q == s_k; scale must be > 0)";
+        case ATTN_ERR_ALIGN: return "misaligned pointer (q/k/v/o need 16 bytes, lse 4 bytes)";
+        case ATTN_ERR_CUDA: return "CUDA runtime or driver error";
+        case ATTN_ERR_TIMEOUT: return "a kernel gave up a bounded device-side wait";
+        default: return "unknown status code";
+    }
+}
+
+extern "C" int attn_set_wait_timeout_ns(uint64_t ns) {
+    g_timeout_ns = ns ? static_cast<unsigned long long>(ns) : kDefaultTimeoutNs;
+    return ATTN_OK;
+}
+
+extern "C" int attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    DeviceState* st = nullptr;
+    int rc = init_device(dev, &st);
+    if (rc != ATTN_OK) return rc;
+    wait_timeout_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+        st->status, static_cast<unsigned long long>(timeout_ns));
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
+extern "C" int attn_last_launch_count(void) { return g_last_launches; }

@@ -1,0 +1,139 @@
+"""CPU tests of the C ABI: the library loads, exports every declared symbol,
+and rejects bad arguments before making any CUDA call."""
+from __future__ import annotations
+
+import ctypes
+import glob
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+from scaled_dot_product_10_b200 import attn
+from scaled_dot_product_10_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return attn.load_library()
+
+
+def declared_functions():
+    names = []
+    for h in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(h).read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        names += re.findall(r"^\s*(?:const\s+)?\w+[\s\*]+(attn_\w+)\s*\(", text, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_entry_points():
+    names = declared_functions()
+    assert "attn_fwd" in names and "attn_status" in names and "attn_strerror" in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), f"{name} declared in include/ but not exported"
+    assert set(declared_functions()) <= set(attn.EXPORTED)
+
+
+def test_strerror(lib):
+    for code in range(6):
+        assert attn.attn_strerror(code)
+    assert "unknown" in attn.attn_strerror(99)
+
+
+# Fake device addresses: validation rejects the call before any CUDA use, so
+# these are never dereferenced.
+A = 0x10000
+
+
+def call(lib, q=A, k=A, v=A, o=None, lse=None, b=1, hq=2, hkv=2, sq=256, sk=256, d=128,
+         causal=0, scale=0.088):
+    o = A if o is None else o
+    lse = A if lse is None else lse
+    return lib.attn_fwd(q, k, v, o, lse, b, hq, hkv, sq, sk, d, causal, scale, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=0), attn.ATTN_ERR_INVALID),
+    (dict(k=0), attn.ATTN_ERR_INVALID),
+    (dict(v=0), attn.ATTN_ERR_INVALID),
+    (dict(o=0), attn.ATTN_ERR_INVALID),
+    (dict(lse=0), attn.ATTN_ERR_INVALID),
+    (dict(b=0), attn.ATTN_ERR_INVALID),
+    (dict(hq=-1), attn.ATTN_ERR_INVALID),
+    (dict(sk=0), attn.ATTN_ERR_INVALID),
+    (dict(hq=6, hkv=4), attn.ATTN_ERR_INVALID),
+    (dict(d=64), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(d=256), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(causal=1, sq=256, sk=512), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(causal=2), attn.ATTN_ERR_INVALID),
+    (dict(scale=float("nan")), attn.ATTN_ERR_INVALID),
+    (dict(scale=float("inf")), attn.ATTN_ERR_INVALID),
+    (dict(scale=0.0), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(scale=-0.1), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(q=A + 8), attn.ATTN_ERR_ALIGN),
+    (dict(k=A + 4), attn.ATTN_ERR_ALIGN),
+    (dict(v=A + 2), attn.ATTN_ERR_ALIGN),
+    (dict(o=A + 8), attn.ATTN_ERR_ALIGN),
+    (dict(lse=A + 2), attn.ATTN_ERR_ALIGN),
+    (dict(b=1 << 20, hq=1 << 10, hkv=1 << 10, sq=1 << 20, sk=128), attn.ATTN_ERR_INVALID),
+])
+def test_validation_codes(lib, kw, code):
+    assert call(lib, **kw) == code
+
+
+def test_error_writes_nothing(lib):
+    o = np.full(64, 7, dtype=np.uint16)
+    lse = np.full(16, 3.0, dtype=np.float32)
+    rc = call(lib, o=o.ctypes.data, lse=lse.ctypes.data, d=64)
+    assert rc == attn.ATTN_ERR_UNSUPPORTED
+    assert np.all(o == 7) and np.all(lse == 3.0)
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
+def test_no_device_reports_cuda_error(lib):
+    assert call(lib) == attn.ATTN_ERR_CUDA
+
+
+def test_host_workspace_bytes(lib):
+    b, hq, hkv, s = 2, 4, 2, 300
+    q = b * s * hq * 128 * 2
+    kv = b * s * hkv * 128 * 2
+    l = b * hq * s * 4
+    r = lambda x: (x + 255) // 256 * 256
+    assert lib.attn_fwd_host_workspace_bytes(b, hq, hkv, s, s, 128) == 2 * r(q) + 2 * r(kv) + r(l)
+    assert lib.attn_fwd_host_workspace_bytes(b, hq, hkv, s, s, 64) == 0
+    assert lib.attn_fwd_host_workspace_bytes(b, 3, 2, s, s, 128) == 0
+
+
+def test_host_entry_validation(lib):
+    args = (A, A, A, A, A, 1, 2, 2, 256, 256, 128, 0, 0.088)
+    need = lib.attn_fwd_host_workspace_bytes(1, 2, 2, 256, 256, 128)
+    assert lib.attn_fwd_host(*args, None, need, None) == attn.ATTN_ERR_INVALID
+    assert lib.attn_fwd_host(*args, A, need - 1, None) == attn.ATTN_ERR_INVALID
+    assert lib.attn_fwd_host(*args, A + 16, need, None) == attn.ATTN_ERR_ALIGN
+
+
+def test_python_binding_rejects_wrong_dtype():
+    q = torch.zeros(1, 8, 2, 128)
+    with pytest.raises(TypeError):
+        attn.attn_fwd(q, q, q)
+
+
+def test_python_binding_requires_cuda_tensors():
+    q = torch.zeros(1, 8, 2, 128, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        attn.attn_fwd(q, q, q)
+
+
+def test_missing_library_fails_loudly(tmp_path):
+    with pytest.raises(OSError):
+        attn.load_library(str(tmp_path / "nope.so"))

@@ -1,0 +1,163 @@
+"""GPU parity: the CUDA path against the FP64 oracle on identical seeded
+BF16 inputs (B200 only)."""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from parity import assert_within, check, gather_rows, metrics, run_gpu
+from scaled_dot_product_10_b200 import attn
+from scaled_dot_product_10_b200.workloads import WORKLOADS, make_qkv, sample_rows, workload_qkv
+
+pytestmark = pytest.mark.gpu
+
+SCALE = 1.0 / math.sqrt(128)
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _gpu():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    attn.load_library()
+
+
+# ----------------------------------------------------------------- small cases
+@pytest.mark.parametrize("causal", [False, True])
+def test_tiny_config(causal):
+    w = WORKLOADS["tiny_b1_h2_s256"]
+    q, k, v = workload_qkv(w)
+    check(q, k, v, causal, w.scale, what=f"{w.name} causal={causal}")
+
+
+# Sequence tails (not multiples of the 128-row tile), single rows, one head.
+@pytest.mark.parametrize("s", [1, 2, 64, 127, 128, 129, 200, 255, 383, 640, 1000])
+@pytest.mark.parametrize("causal", [False, True])
+def test_tails(s, causal):
+    q, k, v = make_qkv(1, 1, 1, s, s, seed=2000 + s)
+    check(q, k, v, causal, SCALE, what=f"s={s} causal={causal}")
+
+
+@pytest.mark.parametrize("s_q,s_k", [(1, 300), (300, 1), (128, 1024), (777, 129), (64, 4096)])
+def test_noncausal_rectangular(s_q, s_k):
+    q, k, v = make_qkv(2, 4, 2, s_q, s_k, seed=3000 + s_q + s_k)
+    check(q, k, v, False, SCALE, what=f"s_q={s_q} s_k={s_k}")
+
+
+@pytest.mark.parametrize("h_q,h_kv", [(16, 2), (16, 1), (8, 8), (6, 3), (4, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_head_sharing_small(h_q, h_kv, causal):
+    q, k, v = make_qkv(2, h_q, h_kv, 384, 384, seed=4000 + h_q * 10 + h_kv)
+    check(q, k, v, causal, SCALE, what=f"h_q={h_q} h_kv={h_kv} causal={causal}")
+
+
+@pytest.mark.parametrize("scale", [1e-3, 0.05, 0.5, 2.0])
+def test_scales(scale):
+    q, k, v = make_qkv(1, 2, 2, 512, 512, seed=5000)
+    check(q, k, v, True, scale, what=f"scale={scale}")
+
+
+def test_many_tiles_more_than_sms():
+    # 2 * 8 * 12 = 192 tiles > 148 SMs: exercises the persistent loop and the
+    # reuse of TMEM, barriers and the Q double buffer across tiles.
+    q, k, v = make_qkv(2, 8, 4, 1536, 1536, seed=6000)
+    for causal in (False, True):
+        check(q, k, v, causal, SCALE, what=f"persistent causal={causal}")
+
+
+def test_uniform_distribution_inputs():
+    q, k, v = make_qkv(2, 4, 4, 700, 700, seed=6100, dist="uniform")
+    for causal in (False, True):
+        check(q, k, v, causal, SCALE, what=f"uniform causal={causal}")
+
+
+def test_large_logits_sharp_softmax():
+    # K x 8: scores up to ~90 in magnitude; exercises the rescale path.
+    q, k, v = make_qkv(1, 2, 2, 1024, 1024, seed=6200, k_scale=8.0)
+    for causal in (False, True):
+        check(q, k, v, causal, SCALE, what=f"sharp causal={causal}")
+
+
+def test_identical_v_rows_exact():
+    # The weights of a row sum to one, so identical V rows come back up to
+    # BF16 rounding of O itself.
+    q, k, _ = make_qkv(1, 2, 2, 384, 384, seed=6300)
+    vrow = torch.randn(1, 1, 2, 128).to(torch.bfloat16)
+    v = vrow.expand(1, 384, 2, 128).contiguous()
+    o, _ = run_gpu(q, k, v, False, SCALE)
+    want = vrow.float().expand(1, 384, 2, 128)
+    assert torch.max(torch.abs(o.float().cpu() - want)) <= 2 * 2 ** -8 * want.abs().max()
+
+
+def test_deterministic():
+    q, k, v = make_qkv(2, 4, 2, 1000, 1000, seed=6400)
+    o1, l1 = run_gpu(q, k, v, True, SCALE)
+    o2, l2 = run_gpu(q, k, v, True, SCALE)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+def test_outputs_stay_in_bounds():
+    # o and lse sit inside larger buffers; the guard regions must be untouched.
+    b, h, s = 1, 2, 200
+    q, k, v = make_qkv(b, h, h, s, s, seed=6500)
+    pad = 4096
+    o_buf = torch.full((pad * 2 + b * s * h * 128,), 1234.0, dtype=torch.bfloat16, device="cuda")
+    l_buf = torch.full((pad * 2 + b * h * s,), -7.0, dtype=torch.float32, device="cuda")
+    o = o_buf[pad:pad + b * s * h * 128].view(b, s, h, 128)
+    lse = l_buf[pad:pad + b * h * s].view(b, h, s)
+    attn.attn_fwd(q.cuda(), k.cuda(), v.cuda(), causal=True, scale=SCALE, o=o, lse=lse)
+    assert attn.attn_status() == attn.ATTN_OK
+    assert torch.all(o_buf[:pad] == 1234.0) and torch.all(o_buf[-pad:] == 1234.0)
+    assert torch.all(l_buf[:pad] == -7.0) and torch.all(l_buf[-pad:] == -7.0)
+    o_ref, l_ref, _ = oracle.attn_fwd(q, k, v, True, SCALE)
+    oo, ll = gather_rows(o, lse, None)
+    assert_within(metrics(oo, ll, o_ref, l_ref), "guarded")
+
+
+def test_host_buffer_entry_point():
+    b, hq, hkv, s = 2, 4, 2, 513
+    q, k, v = make_qkv(b, hq, hkv, s, s, seed=6600)
+    qh, kh, vh = q.pin_memory(), k.pin_memory(), v.pin_memory()
+    oh = torch.empty_like(qh).pin_memory()
+    lh = torch.empty((b, hq, s), dtype=torch.float32).pin_memory()
+    ws = torch.empty(attn.host_workspace_bytes(b, hq, hkv, s, s), dtype=torch.uint8, device="cuda")
+    attn.attn_fwd_host(qh, kh, vh, oh, lh, ws, causal=True, scale=SCALE)
+    assert attn.attn_status() == attn.ATTN_OK
+    o_ref, l_ref, _ = oracle.attn_fwd(q, k, v, True, SCALE)
+    oo, ll = gather_rows(oh, lh, None)
+    assert_within(metrics(oo, ll, o_ref, l_ref), "host entry")
+
+
+def test_bounded_wait_reports_timeout_and_context_survives():
+    assert attn.attn_status() == attn.ATTN_OK
+    assert attn.selftest_wait_timeout(50_000_000) == attn.ATTN_OK  # 50 ms
+    assert attn.attn_status() == attn.ATTN_ERR_TIMEOUT
+    assert attn.attn_status() == attn.ATTN_OK  # the word was cleared
+    q, k, v = make_qkv(1, 2, 2, 256, 256, seed=6700)
+    check(q, k, v, False, SCALE, what="after timeout self-test")
+
+
+# ------------------------------------------------------- the workload configs
+def _rows_for(w, n):
+    return sample_rows(w.batch, w.h_q, w.seq, n, seed=w.seed + 7919)
+
+
+FULL = ["mha_b8_h16_s4096", "gqa_b8_h16_kv2_s2048", "mqa_b8_h16_kv1_s2048"]
+SAMPLED = ["mha_b4_h16_s8192", "mha_b2_h16_s16384", "mha_b1_h16_s32768_k3"]
+
+
+@pytest.mark.parametrize("name", FULL + SAMPLED)
+@pytest.mark.parametrize("causal", [False, True])
+def test_workload_configs(name, causal):
+    """Every config at full size, in the launch configuration the bench
+    times; the oracle evaluates 512 sampled query rows per head on the long
+    sequences and 256 per head on the others (always including rows 0, 1,
+    127, 128, 255, 256 and s-1)."""
+    w = WORKLOADS[name]
+    q, k, v = workload_qkv(w)
+    rows = _rows_for(w, 512 if w.sampled else 256)
+    m = check(q, k, v, causal, w.scale, rows=rows, what=f"{name} causal={causal}")
+    print(name, causal, m)
