@@ -122,7 +122,9 @@ class ClockSampler:
         while not self._stop.is_set():
             try:
                 self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
-                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                get = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                    nv.nvmlDeviceGetCurrentClocksThrottleReasons
+                r = get(self._h)
                 for bit, name in self.REASONS.items():
                     if r & bit:
                         self.reasons.add(name)
@@ -194,7 +196,7 @@ def oracle_sample_rate(w, target_s: float, seed_offset: int = 0):
         return float(4 * d * w.seq * rows.size)
 
     def run(n_rows, seed):
-        rows = sample_rows(w.batch, w.h_q, w.seq, n_rows, seed=seed)
+        rows = sample_rows(w.batch, w.h_q, w.seq, n_rows, seed=seed, include_edges=False)
         t0 = time.perf_counter()
         f = 0.0
         for causal in MODES:
@@ -223,7 +225,8 @@ def run_reference(args, world, rank):
     for i in range(args.warmup + args.steps):
         if rows_n is None:
             rows_n = 1
-        rows = sample_rows(w.batch, w.h_q, w.seq, rows_n, seed=w.seed + 100 + i)
+        rows = sample_rows(w.batch, w.h_q, w.seq, rows_n, seed=w.seed + 100 + i,
+                           include_edges=False)
         t0 = time.perf_counter()
         f = 0.0
         for causal in MODES:

@@ -96,22 +96,24 @@ def workload_qkv(w: Workload):
 EDGE_ROWS = (0, 1, 127, 128, 255, 256)
 
 
-def sample_rows(batch: int, h_q: int, s_q: int, n: int, seed: int) -> np.ndarray:
+def sample_rows(batch: int, h_q: int, s_q: int, n: int, seed: int,
+                include_edges: bool = True) -> np.ndarray:
     """Seeded per-(batch, head) sample of ``n`` distinct query rows, sorted.
 
-    Always contains the edge rows (0, 1, 127, 128, 255, 256, s_q-1 where they
-    exist).  Returns int32 [batch, h_q, n'] with n' = min(n, s_q).
+    With ``include_edges`` the sample always contains the edge rows (0, 1,
+    127, 128, 255, 256, s_q-1 where they exist; ``n`` is raised to hold them).
+    Returns int32 [batch, h_q, n'] with n' = min(n, s_q).
     """
-    n = min(n, s_q)
+    fixed = sorted({r for r in EDGE_ROWS if r < s_q} | {s_q - 1}) if include_edges else []
+    n = min(max(n, len(fixed)), s_q)
     rng = np.random.default_rng(seed)
-    fixed = sorted({r for r in EDGE_ROWS if r < s_q} | {s_q - 1})
     out = np.empty((batch, h_q, n), dtype=np.int32)
+    pool = np.setdiff1d(np.arange(s_q), np.array(fixed, dtype=np.int64))
     for b in range(batch):
         for h in range(h_q):
             if n >= s_q:
                 out[b, h] = np.arange(s_q, dtype=np.int32)
                 continue
-            pool = np.setdiff1d(np.arange(s_q), np.array(fixed), assume_unique=False)
             extra = rng.choice(pool, size=n - len(fixed), replace=False)
-            out[b, h] = np.sort(np.concatenate([np.array(fixed), extra])).astype(np.int32)
+            out[b, h] = np.sort(np.concatenate([np.array(fixed, dtype=np.int64), extra])).astype(np.int32)
     return out
