@@ -44,8 +44,10 @@ typedef enum {
                                  or lse not 4-byte aligned */
     ATTN_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (no device,
                                  launch failure, ...) */
-    ATTN_ERR_TIMEOUT = 5      /* a kernel gave up a bounded wait (reported by
+    ATTN_ERR_TIMEOUT = 5,     /* a kernel gave up a bounded wait (reported by
                                  attn_status) */
+    ATTN_ERR_TOO_LARGE = 6    /* attn_fwd_host_static: the problem does not fit
+                                 the library's static device staging area */
 } attn_status_t;
 
 /*
@@ -90,6 +92,40 @@ int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* l
 
 /* Device workspace bytes attn_fwd_host needs for these sizes (0 on bad sizes). */
 size_t attn_fwd_host_workspace_bytes(int batch, int h_q, int h_kv, int s_q, int s_k, int d);
+
+/*
+ * attn_fwd_host_static -- attn_fwd_host for callers that cannot allocate
+ * device memory: instead of a caller-provided workspace it stages q, k, v, o
+ * and lse in a device array that the library itself declares at file scope
+ * (ATTN_STATIC_STAGING_BYTES, held on every GPU that loads the library until
+ * the process exits).  It calls no cudaMalloc/cudaFree or other allocating
+ * routine.  The paper has no counterpart to this entry point: it is a
+ * deployment convenience of this library.
+ *
+ * Who needs it: code that may not allocate on the device at call time -- a
+ * plugin handed only host arrays by an application that owns all device
+ * memory (for example through a framework's caching allocator that must stay
+ * the only allocator), or a caller that cannot afford the device-wide
+ * synchronisation a cudaMalloc/cudaFree can imply.
+ *
+ *   q, k, v, o, lse   host pointers, layouts of attn_fwd (pinned memory makes
+ *                     the copies asynchronous)
+ *   returns           ATTN_ERR_TOO_LARGE, before any CUDA call, when
+ *                     attn_fwd_host_workspace_bytes(...) exceeds
+ *                     ATTN_STATIC_STAGING_BYTES; otherwise as attn_fwd_host
+ *
+ * The first call on a device looks up the staging array's device address
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.  Every call on a device shares the one staging
+ * array and it keeps the last call's contents; nothing in it needs to start
+ * at zero (each call overwrites the inputs and the kernel writes every output
+ * element).  Calls whose GPU work overlaps -- on different streams, or from
+ * different host threads -- race on the array: serialise them.
+ */
+#define ATTN_STATIC_STAGING_BYTES ((size_t)32 << 20)
+int attn_fwd_host_static(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int batch, int h_q, int h_kv, int s_q, int s_k, int d,
+                         int causal, float scale, void* stream);
 
 /*
  * attn_status -- synchronise `stream`, then read and clear the calling

@@ -16,6 +16,8 @@ ATTN_ERR_UNSUPPORTED = 2
 ATTN_ERR_ALIGN = 3
 ATTN_ERR_CUDA = 4
 ATTN_ERR_TIMEOUT = 5
+ATTN_ERR_TOO_LARGE = 6
+STATIC_STAGING_BYTES = 32 << 20
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_NAME = "libattn_sm100.so"
@@ -29,6 +31,8 @@ _SIGNATURES = [
     ("attn_fwd_host", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
                            _P, ctypes.c_size_t, _P]),
     ("attn_fwd_host_workspace_bytes", ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
+    ("attn_fwd_host_static", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
+                                  _P]),
     ("attn_status", _I, [_P]),
     ("attn_strerror", ctypes.c_char_p, [_I]),
     ("attn_set_wait_timeout_ns", _I, [ctypes.c_uint64]),

@@ -227,6 +227,7 @@ extern "C" const char* attn_strerror(int code) {
         case ATTN_ERR_ALIGN: return "misaligned pointer (q/k/v/o need 16 bytes, lse 4 bytes)";
         case ATTN_ERR_CUDA: return "CUDA runtime or driver error";
         case ATTN_ERR_TIMEOUT: return "a kernel gave up a bounded device-side wait";
+        case ATTN_ERR_TOO_LARGE: return "problem larger than the static device staging area (ATTN_STATIC_STAGING_BYTES)";
         default: return "unknown status code";
     }
 }
@@ -249,3 +250,42 @@ extern "C" int attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream) {
 }
 
 extern "C" int attn_last_launch_count(void) { return g_last_launches; }
+
+// ---------------------------------------------------------------------------
+// attn_fwd_host_static: the host-buffer entry point with its device staging in
+// a file-scope array, for callers that cannot allocate device memory.  Host
+// code must not pass the array's name to a kernel or a copy: on the host it is
+// only a stand-in symbol.  Its device address is looked up once per device.
+namespace {
+
+static __device__ __align__(256) unsigned char g_static_staging[ATTN_STATIC_STAGING_BYTES];
+
+std::mutex g_static_mutex;
+void* g_static_staging_ptr[kMaxDevices] = {};
+
+}  // namespace
+
+extern "C" int attn_fwd_host_static(const void* q, const void* k, const void* v, void* o,
+                                    float* lse, int batch, int h_q, int h_kv, int s_q, int s_k,
+                                    int d, int causal, float scale, void* stream) {
+    int rc = validate(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale);
+    if (rc != ATTN_OK) return rc;
+    const size_t need = attn_fwd_host_workspace_bytes(batch, h_q, h_kv, s_q, s_k, d);
+    if (need > ATTN_STATIC_STAGING_BYTES) return ATTN_ERR_TOO_LARGE;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ERR_CUDA;
+    void* staging = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_static_mutex);
+        if (!g_static_staging_ptr[dev]) {
+            // Set-up, once per device, with that device current.
+            void* ptr = nullptr;
+            if (cudaGetSymbolAddress(&ptr, g_static_staging) != cudaSuccess || !ptr)
+                return ATTN_ERR_CUDA;
+            g_static_staging_ptr[dev] = ptr;
+        }
+        staging = g_static_staging_ptr[dev];
+    }
+    return attn_fwd_host(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale, staging,
+                         ATTN_STATIC_STAGING_BYTES, stream);
+}
