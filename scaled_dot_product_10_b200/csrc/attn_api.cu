@@ -19,7 +19,6 @@ using namespace sdpa10;
 
 constexpr int kKvStages = 4;
 using Layout = SmemLayout<kKvStages>;
-constexpr int kThreads = 192;
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
 // Bytes of K/V that the tiles running at one time should share through L2.
 constexpr size_t kL2SectionBytes = 48ull << 20;
@@ -145,7 +144,8 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
     p.n_qb = (s_q + kBlockM - 1) / kBlockM;
     p.n_kb = (s_k + kBlockN - 1) / kBlockN;
     p.causal = causal;
-    p.num_tiles = batch * h_q * p.n_qb;
+    p.n_pairs = (p.n_qb + 1) / 2;
+    p.num_tiles = batch * h_q * p.n_pairs;
     const size_t unit_bytes = 2ull * s_k * kHeadDim * 2;  // K and V of one (batch, kv head)
     const size_t per_sec = kL2SectionBytes / (unit_bytes ? unit_bytes : 1);
     const int units_total = batch * h_kv;

@@ -1,0 +1,99 @@
+// attn_common.cuh -- constants, launch parameters and the bounded mbarrier
+// waits shared by the attention kernels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "sm100_ptx.cuh"
+
+namespace sdpa10 {
+
+constexpr int kHeadDim = 128;
+constexpr int kBlockM = 128;                        // query rows per tile
+constexpr int kBlockN = 128;                        // keys per key/value tile
+constexpr int kTileBytes = kBlockM * kHeadDim * 2;  // 32 KiB: one Q, K or V tile
+constexpr int kHalfTileBytes = kTileBytes / 2;      // one 64-column (128-byte row) half
+constexpr int kTmemCols = 512;
+constexpr unsigned kStatusTimeout = 1u;
+
+// Rescale the running output only when the row maximum grows by more than
+// this many powers of two; otherwise keep the stale maximum (probabilities
+// then stay below 2^8, well inside FP32 and BF16 range, and the final O / l
+// and LSE are unchanged).
+constexpr float kRescaleThresholdLog2 = 8.0f;
+
+struct FwdParams {
+    int batch, h_q, h_kv, s_q, s_k;
+    int group;    // h_q / h_kv
+    int n_qb;     // ceil(s_q / 128)
+    int n_kb;     // ceil(s_k / 128)
+    int n_pairs;  // ceil(n_qb / 2): CTA tiles per (batch, head)
+    int causal;
+    int num_tiles;
+    int units_per_section;  // (batch, kv head) units whose K/V share L2 at once
+    float scale_log2;       // scale * log2(e)
+    __nv_bfloat16* o;
+    float* lse;
+    unsigned long long timeout_ns;
+    unsigned int* status;
+};
+
+// ------------------------------------------------------------------ waits
+struct WaitCtx {
+    volatile int* abort_flag;  // shared memory, per CTA
+    unsigned int* status;      // global, per device
+    unsigned long long timeout_ns;
+};
+
+// Slow path of a bounded mbarrier wait.  Gives up when the CTA's abort flag
+// is raised (if honoured) or the time limit passes; a timeout raises the
+// abort flag and sets the status word.
+__device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, WaitCtx w,
+                                       bool honour_abort) {
+    const uint64_t t0 = ptx::globaltimer_ns();
+    for (uint32_t i = 1;; ++i) {
+        if (ptx::mbar_try_wait(bar, parity)) return true;
+        if ((i & 31u) == 0) {
+            if (honour_abort && *w.abort_flag) return false;
+            if (ptx::globaltimer_ns() - t0 > w.timeout_ns || i > (1u << 28)) {
+                *w.abort_flag = 1;
+                atomicOr(w.status, kStatusTimeout);
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ bool wait_bar(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+    if (ptx::mbar_try_wait(bar, parity)) return true;
+    return wait_slow(bar, parity, w, true);
+}
+
+
+// Warp-uniform wait: every lane waits, and the warp proceeds only if all did.
+__device__ __forceinline__ bool wait_bar_warp(uint32_t bar, uint32_t parity, const WaitCtx& w) {
+    const bool ok = wait_bar(bar, parity, w);
+    return __all_sync(0xffffffffu, ok);
+}
+
+// Waits on a barrier nothing arrives on; the bounded wait must give up,
+// set the status word and let the kernel return.
+__global__ void wait_timeout_selftest_kernel(unsigned int* status, unsigned long long timeout_ns) {
+    __shared__ __align__(8) uint64_t bar_storage;
+    __shared__ int abort_storage;
+    const uint32_t b = ptx::smem_u32(&bar_storage);
+    if (threadIdx.x == 0) {
+        ptx::mbar_init(b, 1);
+        abort_storage = 0;
+        ptx::fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const WaitCtx w{&abort_storage, status, timeout_ns};
+        wait_bar(b, 0, w);
+    }
+    __syncthreads();
+}
+
+}  // namespace sdpa10
