@@ -26,6 +26,8 @@
 //   warp  8    tcgen05.mma issuer (one lane) and TMEM allocator
 //   warp  9    TMA producer (one lane)
 //   warps 10-11 idle (they complete the control warpgroup for setmaxnreg)
+// One lane issues every MMA in the fixed order P0 V, Q0 K, P1 V, Q1 K, which
+// keeps the two blocks half a period apart.
 // The two warpgroups alternate: while one works through its block's
 // exponentials, the tensor core computes the other block's P V and next
 // Q K^T ("ping-pong"), so neither the tensor pipe nor the exponential unit
@@ -45,13 +47,20 @@
 namespace sdpa10 {
 
 constexpr int kThreads = 384;
-constexpr int kMmaWarp = 8;
+constexpr int kMmaWarp0 = 8;  // issues every MMA, allocates TMEM
 constexpr int kLoadWarp = 9;
+// Exponentials of unmasked blocks: in every 16 column pairs of a 32-key
+// chunk, pairs with index below kPolyPairs go to the FMA-pipe polynomial,
+// the rest to the MUFU ex2 unit, so neither unit alone sets the pace.
+#ifndef SDPA10_POLY_PAIRS
+#define SDPA10_POLY_PAIRS 0
+#endif
+constexpr int kPolyPairs = SDPA10_POLY_PAIRS;
 // Register split (per thread): launched at 65536 / 384 -> 168; the control
-// warpgroup (MMA, TMA and two idle warps) drops to 56 so each softmax
-// warpgroup can rise to 224: 2 * 128 * 224 + 128 * 56 = 384 * 168.
-constexpr uint32_t kRegsSoftmax = 216;
-constexpr uint32_t kRegsControl = 72;
+// warpgroup (MMA, TMA and two idle warps) drops to 88 so each softmax
+// warpgroup can rise to 208: 2 * 128 * 208 + 128 * 88 = 384 * 168.
+constexpr uint32_t kRegsSoftmax = 208;
+constexpr uint32_t kRegsControl = 88;
 
 // ------------------------------------------------------------------ schedule
 // Pair index t -> (batch, query head, first query block).  Pairs are grouped
@@ -111,6 +120,36 @@ struct SmemLayout {
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
+// ------------------------------------------------------------------ exp2 on the FMA pipe
+// 2^x for a pair of FP32 values without the MUFU unit (Cody-Waite style range
+// reduction): x = k + f with k = round(x) and f in [-1/2, 1/2]; 2^f by a
+// degree-3 polynomial whose coefficients are a Remez (minimax relative
+// error) fit of 2^f on [-1/2, 1/2], max relative error 7.5e-5 in FP32 --
+// far below the BF16 rounding P gets next; 2^k enters by adding k to the
+// exponent field.  k comes from adding 1.5 * 2^23, which leaves round(x) in
+// the low mantissa bits.  Inputs below -125 are clamped there (2^-125 ~
+// 2.4e-38 stays a normal number); only unmasked blocks use this path.
+__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
+    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
+    constexpr float c0 = 0.99992805719375610f, c1 = 0.69326096773147583f,
+                    c2 = 0.24261112511157990f, c3 = 0.05517166852951050f;
+    float x0, x1;
+    ptx::f2_unpack(x2, x0, x1);
+    const uint64_t x = ptx::f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+    const uint64_t t = ptx::f2_add(x, ptx::f2_pack(kRound, kRound));     // 1.5*2^23 + k
+    const uint64_t kf = ptx::f2_add(t, ptx::f2_pack(-kRound, -kRound));  // k
+    const uint64_t f = ptx::f2_fma(kf, ptx::f2_pack(-1.f, -1.f), x);     // x - k
+    uint64_t p = ptx::f2_fma(ptx::f2_pack(c3, c3), f, ptx::f2_pack(c2, c2));
+    p = ptx::f2_fma(p, f, ptx::f2_pack(c1, c1));
+    p = ptx::f2_fma(p, f, ptx::f2_pack(c0, c0));
+    float t0, t1, p0, p1;
+    ptx::f2_unpack(t, t0, t1);
+    ptx::f2_unpack(p, p0, p1);
+    const float r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
+    const float r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
+    return ptx::f2_pack(r0, r1);
+}
+
 // ------------------------------------------------------------------ softmax
 // One softmax warpgroup: thread r owns query row r of its block (TMEM lane r).
 template <int KV_STAGES>
@@ -152,7 +191,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
             }
             const int kv0 = j * kBlockN;
             const bool diag = p.causal && (kv0 + kBlockN - 1 > qb * kBlockM);
-            if (diag || kv0 + kBlockN > p.s_k) {
+            const bool masked = diag || kv0 + kBlockN > p.s_k;
+            if (masked) {
                 const int lim_tail = p.s_k - kv0;                           // keys >= s_k
                 const int lim_causal = p.causal ? row - kv0 + 1 : kBlockN;  // keys > row
                 const int lim = min(lim_tail, lim_causal);
@@ -162,17 +202,17 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
             }
             float mx;
             {
-                // Four independent 3-input-max chains, then combine.
-                float m4[4] = {fmaxf(s[0], s[1]), fmaxf(s[2], s[3]), fmaxf(s[4], s[5]),
-                               fmaxf(s[6], s[7])};
+                // Eight independent 3-input-max chains, then combine.
+                float m8[8];
 #pragma unroll
-                for (int k = 8; k < 128; k += 8) {
-                    m4[0] = ptx::max3(m4[0], s[k], s[k + 1]);
-                    m4[1] = ptx::max3(m4[1], s[k + 2], s[k + 3]);
-                    m4[2] = ptx::max3(m4[2], s[k + 4], s[k + 5]);
-                    m4[3] = ptx::max3(m4[3], s[k + 6], s[k + 7]);
+                for (int k = 0; k < 8; ++k) m8[k] = fmaxf(s[2 * k], s[2 * k + 1]);
+#pragma unroll
+                for (int k = 16; k < 128; k += 16) {
+#pragma unroll
+                    for (int t = 0; t < 8; ++t) m8[t] = ptx::max3(m8[t], s[k + 2 * t], s[k + 2 * t + 1]);
                 }
-                mx = ptx::max3(m4[0], m4[1], fmaxf(m4[2], m4[3]));
+                mx = ptx::max3(ptx::max3(m8[0], m8[1], m8[2]), ptx::max3(m8[3], m8[4], m8[5]),
+                               fmaxf(m8[6], m8[7]));
             }
             float alpha = 1.f;
             bool rescale = false;
@@ -214,20 +254,45 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
 
             // P = 2^(s c - m c) in chunks of 32 keys -> 16 packed BF16 columns.
             uint64_t sum2a = ptx::f2_pack(0.f, 0.f), sum2b = sum2a;
+            if (masked) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                uint32_t pk[16];
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t pk[16];
 #pragma unroll
-                for (int k = 0; k < 16; ++k) {
-                    const float p0 = ptx::ex2(fmaf(s[32 * q + 2 * k], c2, neg_mc));
-                    const float p1 = ptx::ex2(fmaf(s[32 * q + 2 * k + 1], c2, neg_mc));
-                    if (k & 1)
-                        sum2b = ptx::f2_add(sum2b, ptx::f2_pack(p0, p1));
-                    else
-                        sum2a = ptx::f2_add(sum2a, ptx::f2_pack(p0, p1));
-                    pk[k] = ptx::pack_bf16x2(p0, p1);
+                    for (int k = 0; k < 16; ++k) {
+                        const uint64_t x = ptx::f2_fma(
+                            ptx::f2_pack(s[32 * q + 2 * k], s[32 * q + 2 * k + 1]), c2x2, nmc2);
+                        float x0, x1;
+                        ptx::f2_unpack(x, x0, x1);
+                        const uint64_t e = ptx::f2_pack(ptx::ex2(x0), ptx::ex2(x1));
+                        if (k & 1) sum2b = ptx::f2_add(sum2b, e);
+                        else sum2a = ptx::f2_add(sum2a, e);
+                        pk[k] = ptx::pack_bf16x2_from(e);
+                    }
+                    ptx::tmem_st16(s_tmem + q * 16, pk);
                 }
-                ptx::tmem_st16(s_tmem + q * 16, pk);
+            } else {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    uint32_t pk[16];
+#pragma unroll
+                    for (int k = 0; k < 16; ++k) {
+                        const uint64_t x = ptx::f2_fma(
+                            ptx::f2_pack(s[32 * q + 2 * k], s[32 * q + 2 * k + 1]), c2x2, nmc2);
+                        uint64_t e;
+                        if (k < kPolyPairs) {
+                            e = exp2_poly_x2(x);
+                        } else {
+                            float x0, x1;
+                            ptx::f2_unpack(x, x0, x1);
+                            e = ptx::f2_pack(ptx::ex2(x0), ptx::ex2(x1));
+                        }
+                        if (k & 1) sum2b = ptx::f2_add(sum2b, e);
+                        else sum2a = ptx::f2_add(sum2a, e);
+                        pk[k] = ptx::pack_bf16x2_from(e);
+                    }
+                    ptx::tmem_st16(s_tmem + q * 16, pk);
+                }
             }
             ptx::tmem_wait_st();
             ptx::tc_fence_before();
@@ -325,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_v);
     }
-    if (warp == kMmaWarp) {
+    if (warp == kMmaWarp0) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
         ptx::tmem_relinquish();
     }
@@ -359,11 +424,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             PairCursor c;
             c.start(p);
             for (; ok && c.valid(p); c.next(p)) {
-                for (int i = 0; i < 2 && ok; ++i) {
-                    if (c.n[i] == 0) continue;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (!ok || c.n[i] == 0) continue;
                     if (!wait_bar(bar(L::bQEmpty + i), (q_loads[i] & 1) ^ 1, wc)) {
                         ok = false;
-                        break;
+                        continue;
                     }
                     const uint32_t dst = sQ + i * kTileBytes;
                     const int row0 = (c.qb0 + i) * kBlockM;
@@ -382,12 +448,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t f = fills - 1 - i;
                 wait_slow(bar(L::bKVFull + f % KV_STAGES), (f / KV_STAGES) & 1, wc, false);
             }
+#pragma unroll
             for (int i = 0; i < 2; ++i)
                 if (q_loads[i] > 0)
                     wait_slow(bar(L::bQFull + i), (q_loads[i] - 1) & 1, wc, false);
         }
         __syncwarp();
-    } else if (warp == kMmaWarp) {
+    } else if (warp == kMmaWarp0) {
         // ============================================================ MMA issuer
         ptx::reg_dealloc<kRegsControl>();
         if (lane == 0) {
@@ -400,20 +467,24 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto wait_fill = [&](uint32_t f) -> bool {
                 return wait_bar(bar(L::bKVFull + f % KV_STAGES), (f / KV_STAGES) & 1, wc);
             };
+            // Descriptor low words (start address >> 4 | leading offset).
+            const uint32_t q_lo = desc_lo_sw128(sQ, 16);
+            const uint32_t k_lo = desc_lo_sw128(sKV, 16);
+            const uint32_t v_lo = desc_lo_sw128(sKV, kHalfTileBytes);
             auto qk = [&](int i, uint32_t kslot) {
-                const uint32_t qa = sQ + i * kTileBytes;
-                const uint32_t ka = sKV + kslot * kTileBytes;
+                const uint32_t qa = q_lo + ((i * kTileBytes) >> 4);
+                const uint32_t ka = k_lo + ((kslot * kTileBytes) >> 4);
 #pragma unroll
                 for (int k = 0; k < kHeadDim / 16; ++k) {
                     // K-major, 128-byte swizzle: 16 BF16 (32 bytes) per step
                     // inside a 64-column half; the second half is 16 KiB on.
-                    const uint32_t off = (k >> 2) * kHalfTileBytes + (k & 3) * 32;
-                    ptx::mma_ss(tmem + i * 128, smem_desc_sw128(qa + off, 16, 1024),
-                                smem_desc_sw128(ka + off, 16, 1024), kIdescQK, k > 0 ? 1u : 0u);
+                    const uint32_t off = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
+                    ptx::mma_ss(tmem + i * 128, desc_from_lo(qa + off), desc_from_lo(ka + off),
+                                kIdescQK, k > 0 ? 1u : 0u);
                 }
             };
             auto pv = [&](int i, uint32_t vslot, bool acc) {
-                const uint32_t va = sKV + vslot * kTileBytes;
+                const uint32_t va = v_lo + ((vslot * kTileBytes) >> 4);
 #pragma unroll
                 for (int k = 0; k < kBlockN / 16; ++k) {
                     // A = P from TMEM: 16 keys = 8 packed columns per step.
@@ -421,7 +492,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // 8-row swizzle atoms = 2 KiB per step; the two 64-wide
                     // head-dim halves are 16 KiB apart (leading offset).
                     ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8,
-                                smem_desc_sw128(va + k * 2048, kHalfTileBytes, 1024), kIdescPV,
+                                desc_from_lo(va + ((k * 2048) >> 4)), kIdescPV,
                                 (acc || k > 0) ? 1u : 0u);
                 }
             };
@@ -429,14 +500,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             c.start(p);
             for (; ok && c.valid(p); c.next(p)) {
                 const int n = c.iters();
-                for (int i = 0; i < 2 && ok; ++i) {
-                    if (c.n[i] == 0) continue;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    if (!ok || c.n[i] == 0) continue;
                     ok = wait_bar(bar(L::bQFull + i), started[i] & 1, wc);
                     ++started[i];
                 }
                 if (!ok || !(ok = wait_fill(fills))) break;
                 ptx::tc_fence_after();
                 const uint32_t k0 = fills % KV_STAGES;
+#pragma unroll
                 for (int i = 0; i < 2; ++i) {
                     if (c.n[i] == 0) continue;
                     qk(i, k0);
@@ -449,6 +522,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const uint32_t fv = fills, fk = fills + 1;
                     const bool has_k = j + 1 < n;
                     bool v_ready = false, k_ready = false;
+#pragma unroll
                     for (int i = 0; i < 2; ++i) {
                         if (j >= c.n[i]) continue;
                         if (!(ok = wait_bar(bar(L::bPFull + i), p_cnt[i] & 1, wc))) break;
@@ -491,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     ptx::tc_fence_before();
     __syncthreads();
-    if (warp == kMmaWarp) {
+    if (warp == kMmaWarp0) {
         ptx::tc_fence_after();
         ptx::tmem_dealloc(tmem, kTmemCols);
     }
