@@ -19,7 +19,7 @@
  * cores; the softmax runs in FP32 (the precision split of the bjdmk.com.cn
  * page, section 3); the probabilities P are rounded to BF16 before the P V
  * product; O is written as BF16 (round to nearest even), LSE as FP32.
- * NaN or Inf in the inputs propagate; they are not checked.
+ * Inputs containing NaN or Inf give unspecified results (not checked).
  *
  * Every function returns an attn_status_t code.  On any error nothing is
  * written to o or lse.
