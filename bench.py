@@ -46,7 +46,7 @@ def parse_args():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="mha_b8_h16_s4096", choices=sorted(WORKLOADS))
     ap.add_argument("--e2e-steps", type=int, default=5)
-    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+    ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -213,9 +213,14 @@ def oracle_sample_rate(w, target_s: float, seed_offset: int = 0):
             f += flops(rows, causal)
         return f, time.perf_counter() - t0
 
-    f1, t1 = run(1, w.seed + 1 + seed_offset)            # calibration
-    per_row = t1 / max(1, w.batch * w.h_q)
-    n = max(1, min(w.seq, int(target_s / max(per_row * w.batch * w.h_q, 1e-9))))
+    # Calibrate t(n) = fixed + per_row * n from two small samples (each call
+    # also pays a fixed cost for decoding the whole inputs), then size the
+    # timed sample to about target_s.
+    _, t1 = run(1, w.seed + 1 + seed_offset)
+    _, t4 = run(4, w.seed + 3 + seed_offset)
+    per_n = max((t4 - t1) / 3.0, 1e-6)
+    fixed = max(t1 - per_n, 0.0)
+    n = max(1, min(w.seq, int((target_s - fixed) / per_n)))
     f, t = run(n, w.seed + 2 + seed_offset)
     return f / t / 1e12, t, n, oracle.num_threads()
 

@@ -1,7 +1,7 @@
 // attn_fwd_kernel.cuh -- fused scaled dot-product attention forward for
-// B200 (sm_100a): TMA -> shared-memory ring -> tcgen05.mma into Tensor
-// Memory -> FP32 online softmax -> tcgen05.mma with P read from Tensor
-// Memory -> BF16 O and FP32 LSE.
+// B200 (sm_100a): TMA -> shared memory -> tcgen05.mma into Tensor Memory ->
+// FP32 online softmax -> P (BF16) in shared memory -> tcgen05.mma -> BF16 O
+// and FP32 LSE.
 //
 // What is computed is the SDPA definition softmax(Q K^T * scale) V (rkmt.cn
 // "GPU attention operator optimisation" page, section 1), evaluated the way
@@ -23,19 +23,29 @@
 //   warps 0-3  softmax warpgroup 0: query block 2p   (TMEM lanes = rows)
 //   warps 4-7  softmax warpgroup 1: query block 2p+1
 //              each also rescales its O when needed and writes its O/LSE
-//   warp  8    tcgen05.mma issuer (one lane) and TMEM allocator
+//   warp  8    tcgen05.mma issuer for query block 0 (one lane); TMEM allocator
 //   warp  9    TMA producer (one lane)
-//   warps 10-11 idle (they complete the control warpgroup for setmaxnreg)
-// One lane issues every MMA in the fixed order P0 V, Q0 K, P1 V, Q1 K, which
-// keeps the two blocks half a period apart.
-// The two warpgroups alternate: while one works through its block's
-// exponentials, the tensor core computes the other block's P V and next
-// Q K^T ("ping-pong"), so neither the tensor pipe nor the exponential unit
-// waits on the other's serial chain.
-// Tensor Memory (512 columns): S0 | S1 | O0 | O1 at columns 0, 128, 256, 384;
-// P_i is written as packed BF16 over the first 64 columns of S_i.
-// Shared memory: Q0, Q1 (32 KiB each) and a KV_STAGES ring of 32 KiB K/V
-// tiles, all in the 128-byte swizzle that TMA writes and tcgen05 reads.
+//   warp 10    tcgen05.mma issuer for query block 1 (one lane)
+//   warp 11    idle (completes the control warpgroup for setmaxnreg)
+// Tensor Memory (512 columns): S0 | S1 | O0 | O1 at columns 0, 128, 256, 384.
+// P_i goes to shared memory (in the layout the MMA reads), so a softmax
+// warpgroup hands S_i back as soon as it has loaded the scores: the next
+// Q K^T of the block then runs while the current exponentials are computed,
+// and the two warpgroups work continuously instead of waiting on their
+// block's P V -> Q K^T chain.  Each block has its own issuing lane, so one
+// block's events never wait behind the other's; a K or V slot is released
+// when both issuers are done with it.
+// The two warpgroups take turns on the exponential unit: their exponential
+// phases run in a fixed global order (per pair, per key block: block 0, then
+// block 1), passed on through a "turn" mbarrier, so one warpgroup's loads,
+// row max and waits overlap the other's exponentials instead of both
+// warpgroups doing the same phase at the same time.
+// Shared memory: Q0, Q1, P0, P1 (32 KiB each), a ring of K_STAGES K tiles and
+// a ring of V_STAGES V tiles (32 KiB each), all in the 128-byte swizzle that
+// TMA writes and tcgen05 reads.  K and V have separate rings: K(j+1) is used
+// early in step j (right after the softmax frees S) and released soon after,
+// while V(j) is held until the end of step j's softmax, so V gets the
+// deeper ring.
 //
 // Every wait is bounded (per-CTA abort flag plus a global-timer limit); a
 // wait that gives up sets the device status word, and the CTA drains its
@@ -47,20 +57,22 @@
 namespace sdpa10 {
 
 constexpr int kThreads = 384;
-constexpr int kMmaWarp0 = 8;  // issues every MMA, allocates TMEM
+constexpr int kMmaWarp0 = 8;   // issues query block 0's MMAs, allocates TMEM
 constexpr int kLoadWarp = 9;
+constexpr int kMmaWarp1 = 10;  // issues query block 1's MMAs
 // Exponentials of unmasked blocks: in every 16 column pairs of a 32-key
 // chunk, pairs with index below kPolyPairs go to the FMA-pipe polynomial,
-// the rest to the MUFU ex2 unit, so neither unit alone sets the pace.
+// the rest to the MUFU ex2 unit.  Measured slower than MUFU alone on B200,
+// so it is off unless SDPA10_POLY_PAIRS is set at build time.
 #ifndef SDPA10_POLY_PAIRS
 #define SDPA10_POLY_PAIRS 0
 #endif
 constexpr int kPolyPairs = SDPA10_POLY_PAIRS;
 // Register split (per thread): launched at 65536 / 384 -> 168; the control
-// warpgroup (MMA, TMA and two idle warps) drops to 88 so each softmax
-// warpgroup can rise to 208: 2 * 128 * 208 + 128 * 88 = 384 * 168.
-constexpr uint32_t kRegsSoftmax = 208;
-constexpr uint32_t kRegsControl = 88;
+// warpgroup (two MMA issuers, TMA, one idle warp) drops to 72 so each softmax
+// warpgroup can rise to 216: 2 * 128 * 216 + 128 * 72 = 384 * 168.
+constexpr uint32_t kRegsSoftmax = 216;
+constexpr uint32_t kRegsControl = 72;
 
 // ------------------------------------------------------------------ schedule
 // Pair index t -> (batch, query head, first query block).  Pairs are grouped
@@ -106,14 +118,21 @@ struct PairCursor {
 };
 
 // ------------------------------------------------------------------ layout
-template <int KV_STAGES>
+constexpr int K_STAGES = 1;
+constexpr int V_STAGES = 2;
+template <int K_STAGES_>
 struct SmemLayout {
-    static constexpr int kQ = 0;                                // Q0, Q1
-    static constexpr int kKV = 2 * kTileBytes;                  // ring
-    static constexpr int kBars = kKV + KV_STAGES * kTileBytes;  // mbarriers
-    static constexpr int bQFull = 0, bQEmpty = 2, bKVFull = 4, bKVEmpty = 4 + KV_STAGES,
-                         bSFull = 4 + 2 * KV_STAGES, bPFull = bSFull + 2, bOFull = bPFull + 2,
-                         bOEmpty = bOFull + 2, bDrain = bOEmpty + 2, kNumBars = bDrain + 1;
+    static constexpr int kQ = 0;                              // Q0, Q1
+    static constexpr int kP = 2 * kTileBytes;                 // P0, P1
+    static constexpr int kK = 4 * kTileBytes;                 // K ring
+    static constexpr int kV = kK + K_STAGES * kTileBytes;     // V ring
+    static constexpr int kBars = kV + V_STAGES * kTileBytes;  // mbarriers
+    static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = 4 + K_STAGES,
+                         bVFull = 4 + 2 * K_STAGES, bVEmpty = bVFull + V_STAGES,
+                         bSFull = bVEmpty + V_STAGES,
+                         bSFree = bSFull + 2, bPFull = bSFree + 2, bOFull = bPFull + 2,
+                         bOEmpty = bOFull + 2, bTurn = bOEmpty + 2, bDrain = bTurn + 1,
+                         kNumBars = bDrain + 2;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
@@ -152,26 +171,36 @@ __device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
 
 // ------------------------------------------------------------------ softmax
 // One softmax warpgroup: thread r owns query row r of its block (TMEM lane r).
-template <int KV_STAGES>
+template <int K_STAGES>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& wc,
-                                             uint32_t tmem, uint32_t bars, int wg, int warp_in_wg,
-                                             int lane) {
-    using L = SmemLayout<KV_STAGES>;
+                                             uint32_t tmem, uint32_t sP, uint32_t bars, int wg,
+                                             int warp_in_wg, int lane) {
+    using L = SmemLayout<K_STAGES>;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
     const int r = warp_in_wg * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(warp_in_wg * 32) << 16;
     const uint32_t s_tmem = tmem + lane_base + wg * 128;
     const uint32_t o_tmem = tmem + lane_base + 256 + wg * 128;
-    const uint32_t b_sfull = bar(L::bSFull + wg), b_pfull = bar(L::bPFull + wg);
+    const uint32_t b_sfull = bar(L::bSFull + wg), b_sfree = bar(L::bSFree + wg);
+    const uint32_t b_pfull = bar(L::bPFull + wg);
     const uint32_t b_ofull = bar(L::bOFull + wg), b_oempty = bar(L::bOEmpty + wg);
+    // This row of P in shared memory (K-major, 128-byte swizzle, two 64-key
+    // halves 16 KiB apart): 16-byte chunk c of the row lands at
+    // row_base + (c / 8) * 16 KiB + ((c % 8) ^ (r % 8)) * 16.
+    const uint32_t p_row = sP + wg * kTileBytes + (r >> 3) * 1024 + (r & 7) * 128;
+    const uint32_t p_xor = static_cast<uint32_t>(r & 7);
     const float c2 = p.scale_log2;
     const uint64_t c2x2 = ptx::f2_pack(c2, c2);
 
-    uint32_t cnt = 0;  // S blocks this warpgroup has processed (all pairs)
+    const uint32_t b_turn = bar(L::bTurn);
+    uint32_t cnt = 0;   // S blocks this warpgroup has processed (all pairs)
+    uint32_t seq0 = 0;  // exponential phases of both warpgroups before this pair
     PairCursor c;
     c.start(p);
     for (; c.valid(p); c.next(p)) {
         const int n = c.n[wg];
+        const uint32_t seq = seq0;
+        seq0 += static_cast<uint32_t>(c.n[0] + c.n[1]);
         if (n == 0) continue;
         const int qb = c.qb0 + wg;
         const int row = qb * kBlockM + r;
@@ -189,6 +218,11 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
 #pragma unroll
                 for (int k = 0; k < 128; ++k) s[k] = __uint_as_float(sr[k >> 5][k & 31]);
             }
+            // The scores are in registers: S_i may take the next Q K^T.
+            ptx::tc_fence_before();
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(b_sfree);
+
             const int kv0 = j * kBlockN;
             const bool diag = p.causal && (kv0 + kBlockN - 1 > qb * kBlockM);
             const bool masked = diag || kv0 + kBlockN > p.s_k;
@@ -227,9 +261,11 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
             const float neg_mc = -m_ref * c2;
             const uint64_t nmc2 = ptx::f2_pack(neg_mc, neg_mc);
 
-            // Correction: O *= alpha once the previous P V has landed.
+            // The previous P V of this block must be done before its P
+            // buffer is rewritten (and before O is rescaled).
+            if (cnt > 0 && !wait_bar_warp(b_ofull, (cnt - 1) & 1, wc)) return;
             if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-                if (!wait_bar_warp(b_ofull, (cnt - 1) & 1, wc)) return;
+                // Correction: O *= alpha.
                 ptx::tc_fence_after();
                 const uint64_t a2 = ptx::f2_pack(alpha, alpha);
 #pragma unroll
@@ -250,54 +286,46 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
                     ptx::tmem_st32(o_tmem + q * 32, ov);
                 }
                 ptx::tmem_wait_st();
+                ptx::tc_fence_before();
             }
 
-            // P = 2^(s c - m c) in chunks of 32 keys -> 16 packed BF16 columns.
+            // Our turn on the exponential unit: phase index m in the global
+            // order (block 0 before block 1 at each key block j).
+            const uint32_t m = wg == 0 ? seq + j + min(j, c.n[1])
+                                       : seq + min(j + 1, c.n[0]) + j;
+            if (m > 0 && !wait_bar_warp(b_turn, (m - 1) & 1, wc)) return;
+            // P = 2^(s c - m c), 8 keys -> one 16-byte chunk of the P row.
             uint64_t sum2a = ptx::f2_pack(0.f, 0.f), sum2b = sum2a;
-            if (masked) {
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t pk[16];
+            for (int cc = 0; cc < 16; ++cc) {
+                uint32_t w[4];
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const uint64_t x = ptx::f2_fma(
-                            ptx::f2_pack(s[32 * q + 2 * k], s[32 * q + 2 * k + 1]), c2x2, nmc2);
+                for (int k = 0; k < 4; ++k) {
+                    const int e0 = 8 * cc + 2 * k;
+                    const uint64_t x = ptx::f2_fma(ptx::f2_pack(s[e0], s[e0 + 1]), c2x2, nmc2);
+                    uint64_t e;
+                    if (kPolyPairs > 0 && !masked && ((cc * 4 + k) & 15) < kPolyPairs) {
+                        e = exp2_poly_x2(x);
+                    } else {
                         float x0, x1;
                         ptx::f2_unpack(x, x0, x1);
-                        const uint64_t e = ptx::f2_pack(ptx::ex2(x0), ptx::ex2(x1));
-                        if (k & 1) sum2b = ptx::f2_add(sum2b, e);
-                        else sum2a = ptx::f2_add(sum2a, e);
-                        pk[k] = ptx::pack_bf16x2_from(e);
+                        e = ptx::f2_pack(ptx::ex2(x0), ptx::ex2(x1));
                     }
-                    ptx::tmem_st16(s_tmem + q * 16, pk);
+                    if (k & 1) sum2b = ptx::f2_add(sum2b, e);
+                    else sum2a = ptx::f2_add(sum2a, e);
+                    w[k] = ptx::pack_bf16x2_from(e);
                 }
-            } else {
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t pk[16];
-#pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const uint64_t x = ptx::f2_fma(
-                            ptx::f2_pack(s[32 * q + 2 * k], s[32 * q + 2 * k + 1]), c2x2, nmc2);
-                        uint64_t e;
-                        if (k < kPolyPairs) {
-                            e = exp2_poly_x2(x);
-                        } else {
-                            float x0, x1;
-                            ptx::f2_unpack(x, x0, x1);
-                            e = ptx::f2_pack(ptx::ex2(x0), ptx::ex2(x1));
-                        }
-                        if (k & 1) sum2b = ptx::f2_add(sum2b, e);
-                        else sum2a = ptx::f2_add(sum2a, e);
-                        pk[k] = ptx::pack_bf16x2_from(e);
-                    }
-                    ptx::tmem_st16(s_tmem + q * 16, pk);
-                }
+                ptx::st_shared_v4(p_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ p_xor) << 4),
+                                  w[0], w[1], w[2], w[3]);
             }
-            ptx::tmem_wait_st();
-            ptx::tc_fence_before();
+            // P visible to the tensor core (async proxy), then hand it over;
+            // pass the exponential turn on.
+            ptx::fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(b_pfull);
+            if (lane == 0) {
+                ptx::mbar_arrive(b_pfull);
+                ptx::mbar_arrive(b_turn);
+            }
             {
                 float a0, a1, b0, b1;
                 ptx::f2_unpack(sum2a, a0, a1);
@@ -348,18 +376,21 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
 }
 
 // ------------------------------------------------------------------ kernel
-template <int KV_STAGES>
+template <int K_STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
-                          const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-    using L = SmemLayout<KV_STAGES>;
+                          const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ FwdParams p) {
+    using L = SmemLayout<K_STAGES>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
     const uint32_t sbase = ptx::smem_u32(smem);
     const uint32_t sQ = sbase + L::kQ;
-    const uint32_t sKV = sbase + L::kKV;
+    const uint32_t sP = sbase + L::kP;
+    const uint32_t sK = sbase + L::kK;
+    const uint32_t sV = sbase + L::kV;
     const uint32_t bars = sbase + L::kBars;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
@@ -373,14 +404,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(bar(L::bQFull + i), 1);
             ptx::mbar_init(bar(L::bQEmpty + i), 1);
             ptx::mbar_init(bar(L::bSFull + i), 1);
+            ptx::mbar_init(bar(L::bSFree + i), 4);
             ptx::mbar_init(bar(L::bPFull + i), 4);
             ptx::mbar_init(bar(L::bOFull + i), 1);
             ptx::mbar_init(bar(L::bOEmpty + i), 4);
         }
-        for (int i = 0; i < KV_STAGES; ++i) {
-            ptx::mbar_init(bar(L::bKVFull + i), 1);
-            ptx::mbar_init(bar(L::bKVEmpty + i), 1);
+        for (int i = 0; i < K_STAGES; ++i) {
+            ptx::mbar_init(bar(L::bKFull + i), 1);
+            ptx::mbar_init(bar(L::bKEmpty + i), 2);  // one arrival per MMA issuer
         }
+        for (int i = 0; i < V_STAGES; ++i) {
+            ptx::mbar_init(bar(L::bVFull + i), 1);
+            ptx::mbar_init(bar(L::bVEmpty + i), 2);
+        }
+        ptx::mbar_init(bar(L::bDrain + 1), 1);
+        ptx::mbar_init(bar(L::bTurn), 4);  // the 4 warps of the finishing warpgroup
         ptx::mbar_init(bar(L::bDrain), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -406,19 +444,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             const uint64_t pol_kv = ptx::policy_evict_last();
             const uint64_t pol_q = ptx::policy_evict_first();
-            uint32_t fills = 0;         // key/value tiles issued
+            uint32_t k_loads = 0, v_loads = 0;  // K / V tiles issued
             uint32_t q_loads[2] = {0, 0};
             bool ok = true;
-            auto load_kv = [&](const CUtensorMap* tm, const PairCursor& c, int j) -> bool {
-                const int slot = fills % KV_STAGES;
-                if (!wait_bar(bar(L::bKVEmpty + slot), ((fills / KV_STAGES) & 1) ^ 1, wc))
+            auto load_tile = [&](const CUtensorMap* tm, uint32_t dst, uint32_t full, const PairCursor& c,
+                                 int j) {
+                ptx::mbar_arrive_expect_tx(full, kTileBytes);
+                ptx::tma_load_4d(dst, tm, full, 0, c.g, j * kBlockN, c.b, pol_kv);
+                ptx::tma_load_4d(dst + kHalfTileBytes, tm, full, 64, c.g, j * kBlockN, c.b, pol_kv);
+            };
+            auto load_k = [&](const PairCursor& c, int j) -> bool {
+                const int slot = k_loads % K_STAGES;
+                if (!wait_bar(bar(L::bKEmpty + slot), ((k_loads / K_STAGES) & 1) ^ 1, wc))
                     return false;
-                const uint32_t dst = sKV + slot * kTileBytes;
-                ptx::mbar_arrive_expect_tx(bar(L::bKVFull + slot), kTileBytes);
-                ptx::tma_load_4d(dst, tm, bar(L::bKVFull + slot), 0, c.g, j * kBlockN, c.b, pol_kv);
-                ptx::tma_load_4d(dst + kHalfTileBytes, tm, bar(L::bKVFull + slot), 64, c.g,
-                                 j * kBlockN, c.b, pol_kv);
-                ++fills;
+                load_tile(&tm_k, sK + slot * kTileBytes, bar(L::bKFull + slot), c, j);
+                ++k_loads;
+                return true;
+            };
+            auto load_v = [&](const PairCursor& c, int j) -> bool {
+                const int slot = v_loads % V_STAGES;
+                if (!wait_bar(bar(L::bVEmpty + slot), ((v_loads / V_STAGES) & 1) ^ 1, wc))
+                    return false;
+                load_tile(&tm_v, sV + slot * kTileBytes, bar(L::bVFull + slot), c, j);
+                ++v_loads;
                 return true;
             };
             PairCursor c;
@@ -439,14 +487,23 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      row0, c.b, pol_q);
                     ++q_loads[i];
                 }
-                // Issue order = the MMA warp's consumption order: K0 V0 K1 V1 ...
+                // Issue order = the MMA warp's consumption order:
+                // K0, then for each step j: K(j+1), V(j).
                 const int n = c.iters();
-                for (int j = 0; j < n && ok; ++j) ok = load_kv(&tm_k, c, j) && load_kv(&tm_v, c, j);
+                if (ok) ok = load_k(c, 0);
+                for (int j = 0; j < n && ok; ++j) {
+                    if (j + 1 < n) ok = load_k(c, j + 1);
+                    if (ok) ok = load_v(c, j);
+                }
             }
             // Drain: every issued copy must land before the CTA may exit.
-            for (int i = 0; i < KV_STAGES && i < static_cast<int>(fills); ++i) {
-                const uint32_t f = fills - 1 - i;
-                wait_slow(bar(L::bKVFull + f % KV_STAGES), (f / KV_STAGES) & 1, wc, false);
+            for (int i = 0; i < K_STAGES && i < static_cast<int>(k_loads); ++i) {
+                const uint32_t f = k_loads - 1 - i;
+                wait_slow(bar(L::bKFull + f % K_STAGES), (f / K_STAGES) & 1, wc, false);
+            }
+            for (int i = 0; i < V_STAGES && i < static_cast<int>(v_loads); ++i) {
+                const uint32_t f = v_loads - 1 - i;
+                wait_slow(bar(L::bVFull + f % V_STAGES), (f / V_STAGES) & 1, wc, false);
             }
 #pragma unroll
             for (int i = 0; i < 2; ++i)
@@ -454,111 +511,122 @@ __global__ void __launch_bounds__(kThreads, 1)
                     wait_slow(bar(L::bQFull + i), (q_loads[i] - 1) & 1, wc, false);
         }
         __syncwarp();
-    } else if (warp == kMmaWarp0) {
-        // ============================================================ MMA issuer
+    } else if (warp == kMmaWarp0 || warp == kMmaWarp1) {
+        // ============================================================ MMA issuers
         ptx::reg_dealloc<kRegsControl>();
         if (lane == 0) {
+            const int i = (warp == kMmaWarp0) ? 0 : 1;  // query block this lane serves
             constexpr uint32_t kIdescQK = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
             constexpr uint32_t kIdescPV = idesc_bf16_f32(kBlockM, kHeadDim, 0, 1);
-            uint32_t fills = 0;          // key/value tiles consumed
-            uint32_t started[2] = {0, 0};  // pairs in which query block i was active
-            uint32_t p_cnt[2] = {0, 0};  // P blocks consumed
+            uint32_t k_used = 0, v_used = 0;  // K / V tiles passed (used or skipped)
+            uint32_t started = 0;             // pairs in which query block i was active
+            uint32_t s_cnt = 0, pv_cnt = 0;   // Q K^T / P V groups issued
             bool ok = true;
-            auto wait_fill = [&](uint32_t f) -> bool {
-                return wait_bar(bar(L::bKVFull + f % KV_STAGES), (f / KV_STAGES) & 1, wc);
-            };
             // Descriptor low words (start address >> 4 | leading offset).
-            const uint32_t q_lo = desc_lo_sw128(sQ, 16);
-            const uint32_t k_lo = desc_lo_sw128(sKV, 16);
-            const uint32_t v_lo = desc_lo_sw128(sKV, kHalfTileBytes);
-            auto qk = [&](int i, uint32_t kslot) {
-                const uint32_t qa = q_lo + ((i * kTileBytes) >> 4);
-                const uint32_t ka = k_lo + ((kslot * kTileBytes) >> 4);
+            const uint32_t q_lo = desc_lo_sw128(sQ + i * kTileBytes, 16);
+            const uint32_t p_lo = desc_lo_sw128(sP + i * kTileBytes, 16);
+            const uint32_t k_lo = desc_lo_sw128(sK, 16);
+            const uint32_t v_lo = desc_lo_sw128(sV, kHalfTileBytes);
+            const uint32_t s_tm = tmem + i * 128, o_tm = tmem + 256 + i * 128;
+            auto wait_k = [&]() -> bool {
+                return wait_bar(bar(L::bKFull + k_used % K_STAGES), (k_used / K_STAGES) & 1, wc);
+            };
+            auto wait_v = [&]() -> bool {
+                return wait_bar(bar(L::bVFull + v_used % V_STAGES), (v_used / V_STAGES) & 1, wc);
+            };
+            // A tile this block does not use: once it has landed (so the slot's
+            // previous use is released), give up this issuer's share of it.
+            auto skip_k = [&]() -> bool {
+                if (!wait_k()) return false;
+                ptx::mbar_arrive(bar(L::bKEmpty + k_used % K_STAGES));
+                ++k_used;
+                return true;
+            };
+            auto skip_v = [&]() -> bool {
+                if (!wait_v()) return false;
+                ptx::mbar_arrive(bar(L::bVEmpty + v_used % V_STAGES));
+                ++v_used;
+                return true;
+            };
+            // S_i = Q_i K^T once warpgroup i has read its previous S.
+            auto qk = [&](bool last_of_pair) -> bool {
+                if (!wait_k()) return false;
+                if (s_cnt > 0 && !wait_bar(bar(L::bSFree + i), (s_cnt - 1) & 1, wc)) return false;
+                ptx::tc_fence_after();
+                const uint32_t ka = k_lo + (((k_used % K_STAGES) * kTileBytes) >> 4);
 #pragma unroll
                 for (int k = 0; k < kHeadDim / 16; ++k) {
                     // K-major, 128-byte swizzle: 16 BF16 (32 bytes) per step
                     // inside a 64-column half; the second half is 16 KiB on.
                     const uint32_t off = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
-                    ptx::mma_ss(tmem + i * 128, desc_from_lo(qa + off), desc_from_lo(ka + off),
-                                kIdescQK, k > 0 ? 1u : 0u);
+                    ptx::mma_ss(s_tm, desc_from_lo(q_lo + off), desc_from_lo(ka + off), kIdescQK,
+                                k > 0 ? 1u : 0u);
                 }
+                ptx::mma_commit(bar(L::bSFull + i));
+                if (last_of_pair) ptx::mma_commit(bar(L::bQEmpty + i));
+                ptx::mma_commit(bar(L::bKEmpty + k_used % K_STAGES));
+                ++k_used;
+                ++s_cnt;
+                return true;
             };
-            auto pv = [&](int i, uint32_t vslot, bool acc) {
-                const uint32_t va = v_lo + ((vslot * kTileBytes) >> 4);
+            // O_i += P_i V once P_i is in shared memory.
+            auto pv = [&](bool acc) -> bool {
+                if (!wait_v()) return false;
+                if (!wait_bar(bar(L::bPFull + i), pv_cnt & 1, wc)) return false;
+                ptx::tc_fence_after();
+                const uint32_t va = v_lo + (((v_used % V_STAGES) * kTileBytes) >> 4);
 #pragma unroll
                 for (int k = 0; k < kBlockN / 16; ++k) {
-                    // A = P from TMEM: 16 keys = 8 packed columns per step.
-                    // B = V, MN-major (head dim contiguous): 16 keys = two
-                    // 8-row swizzle atoms = 2 KiB per step; the two 64-wide
-                    // head-dim halves are 16 KiB apart (leading offset).
-                    ptx::mma_ts(tmem + 256 + i * 128, tmem + i * 128 + k * 8,
+                    // A = P (K-major like Q); B = V, MN-major (head dim
+                    // contiguous): 16 keys = two 8-row swizzle atoms = 2 KiB
+                    // per step; the two 64-wide head-dim halves are 16 KiB apart.
+                    const uint32_t off = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
+                    ptx::mma_ss(o_tm, desc_from_lo(p_lo + off),
                                 desc_from_lo(va + ((k * 2048) >> 4)), kIdescPV,
                                 (acc || k > 0) ? 1u : 0u);
                 }
+                ptx::mma_commit(bar(L::bOFull + i));
+                ptx::mma_commit(bar(L::bVEmpty + v_used % V_STAGES));
+                ++v_used;
+                ++pv_cnt;
+                return true;
             };
             PairCursor c;
             c.start(p);
             for (; ok && c.valid(p); c.next(p)) {
                 const int n = c.iters();
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    if (!ok || c.n[i] == 0) continue;
-                    ok = wait_bar(bar(L::bQFull + i), started[i] & 1, wc);
-                    ++started[i];
+                const int ni = c.n[i];
+                // Tile order (the producer's): K0, then per step j: K(j+1), V(j).
+                if (ni > 0) {
+                    if (!(ok = wait_bar(bar(L::bQFull + i), started & 1, wc))) break;
+                    ++started;
+                    if (!(ok = qk(ni == 1))) break;
+                } else if (!(ok = skip_k())) {
+                    break;
                 }
-                if (!ok || !(ok = wait_fill(fills))) break;
-                ptx::tc_fence_after();
-                const uint32_t k0 = fills % KV_STAGES;
-#pragma unroll
-                for (int i = 0; i < 2; ++i) {
-                    if (c.n[i] == 0) continue;
-                    qk(i, k0);
-                    ptx::mma_commit(bar(L::bSFull + i));
-                    if (c.n[i] == 1) ptx::mma_commit(bar(L::bQEmpty + i));
-                }
-                ptx::mma_commit(bar(L::bKVEmpty + k0));
-                ++fills;
                 for (int j = 0; j < n && ok; ++j) {
-                    const uint32_t fv = fills, fk = fills + 1;
-                    const bool has_k = j + 1 < n;
-                    bool v_ready = false, k_ready = false;
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) {
-                        if (j >= c.n[i]) continue;
-                        if (!(ok = wait_bar(bar(L::bPFull + i), p_cnt[i] & 1, wc))) break;
-                        ++p_cnt[i];
-                        // O_i is free once the previous pair's epilogue read it.
-                        if (j == 0 && started[i] > 1 &&
-                            !(ok = wait_bar(bar(L::bOEmpty + i), started[i] & 1, wc)))
-                            break;
-                        if (!v_ready && !(ok = wait_fill(fv))) break;
-                        v_ready = true;
-                        ptx::tc_fence_after();
-                        pv(i, fv % KV_STAGES, j > 0);
-                        ptx::mma_commit(bar(L::bOFull + i));
-                        if (j + 1 < c.n[i]) {
-                            if (!k_ready && !(ok = wait_fill(fk))) break;
-                            k_ready = true;
-                            ptx::tc_fence_after();
-                            qk(i, fk % KV_STAGES);
-                            ptx::mma_commit(bar(L::bSFull + i));
-                            if (j + 2 == c.n[i]) ptx::mma_commit(bar(L::bQEmpty + i));
-                        }
-                    }
+                    // Next scores first: they are what the softmax waits for.
+                    if (j + 1 < n) ok = (j + 1 < ni) ? qk(j + 2 == ni) : skip_k();
                     if (!ok) break;
-                    ptx::mma_commit(bar(L::bKVEmpty + fv % KV_STAGES));
-                    if (has_k) ptx::mma_commit(bar(L::bKVEmpty + fk % KV_STAGES));
-                    fills += has_k ? 2 : 1;
+                    if (j < ni) {
+                        // O_i is free once the previous pair's epilogue read it.
+                        if (j == 0 && started > 1 &&
+                            !(ok = wait_bar(bar(L::bOEmpty + i), started & 1, wc)))
+                            break;
+                        ok = pv(j > 0);
+                    } else {
+                        ok = skip_v();
+                    }
                 }
             }
             // Drain: all issued MMAs complete before Tensor Memory is freed.
-            ptx::mma_commit(bar(L::bDrain));
-            wait_slow(bar(L::bDrain), 0, wc, false);
+            ptx::mma_commit(bar(L::bDrain + i));
+            wait_slow(bar(L::bDrain + i), 0, wc, false);
         }
         __syncwarp();
     } else if (warp < 8) {
         ptx::reg_alloc<kRegsSoftmax>();
-        softmax_role<KV_STAGES>(p, wc, tmem, bars, warp >> 2, warp & 3, lane);
+        softmax_role<K_STAGES>(p, wc, tmem, sP, bars, warp >> 2, warp & 3, lane);
     } else {
         ptx::reg_dealloc<kRegsControl>();  // idle warps of the control warpgroup
     }
