@@ -51,16 +51,18 @@ struct WaitCtx {
 // abort flag and sets the status word.
 __device__ __forceinline__ bool wait_slow(uint32_t bar, uint32_t parity, WaitCtx w,
                                        bool honour_abort) {
+    // Each probe may sleep up to kSuspendNs in hardware (woken as soon as
+    // the phase completes); the abort flag and the time limit are checked
+    // after every probe, so the wait stays bounded.
+    constexpr uint32_t kSuspendNs = 20000;
     const uint64_t t0 = ptx::globaltimer_ns();
     for (uint32_t i = 1;; ++i) {
-        if (ptx::mbar_try_wait(bar, parity)) return true;
-        if ((i & 31u) == 0) {
-            if (honour_abort && *w.abort_flag) return false;
-            if (ptx::globaltimer_ns() - t0 > w.timeout_ns || i > (1u << 28)) {
-                *w.abort_flag = 1;
-                atomicOr(w.status, kStatusTimeout);
-                return false;
-            }
+        if (ptx::mbar_try_wait_sleep(bar, parity, kSuspendNs)) return true;
+        if (honour_abort && *w.abort_flag) return false;
+        if (ptx::globaltimer_ns() - t0 > w.timeout_ns || i > (1u << 28)) {
+            *w.abort_flag = 1;
+            atomicOr(w.status, kStatusTimeout);
+            return false;
         }
     }
 }

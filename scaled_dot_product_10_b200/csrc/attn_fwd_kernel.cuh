@@ -318,14 +318,13 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
                 ptx::st_shared_v4(p_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ p_xor) << 4),
                                   w[0], w[1], w[2], w[3]);
             }
-            // P visible to the tensor core (async proxy), then hand it over;
-            // pass the exponential turn on.
+            // The exponentials are done: pass the turn on first, then make P
+            // visible to the tensor core (async proxy) and hand it over.
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(b_turn);
             ptx::fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                ptx::mbar_arrive(b_pfull);
-                ptx::mbar_arrive(b_turn);
-            }
+            if (lane == 0) ptx::mbar_arrive(b_pfull);
             {
                 float a0, a1, b0, b1;
                 ptx::f2_unpack(sum2a, a0, a1);
