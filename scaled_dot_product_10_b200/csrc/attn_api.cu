@@ -17,8 +17,7 @@ namespace {
 
 using namespace sdpa10;
 
-constexpr int kKStages = 1;
-using Layout = SmemLayout<kKStages>;
+using Layout = SmemLayout;
 constexpr unsigned long long kDefaultTimeoutNs = 2000000000ull;
 // Bytes of K/V that the tiles running at one time should share through L2.
 constexpr size_t kL2SectionBytes = 48ull << 20;
@@ -56,7 +55,7 @@ int init_device(int dev, DeviceState** out) {
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return ATTN_ERR_CUDA;
-        if (cudaFuncSetAttribute(attn_fwd_sm100_kernel<kKStages>,
+        if (cudaFuncSetAttribute(attn_fwd_sm100_kernel,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Layout::kAlloc) != cudaSuccess)
             return ATTN_ERR_CUDA;
@@ -157,7 +156,7 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
     p.status = st->status;
 
     const int grid = p.num_tiles < st->num_sms ? p.num_tiles : st->num_sms;
-    attn_fwd_sm100_kernel<kKStages><<<grid, kThreads, Layout::kAlloc,
+    attn_fwd_sm100_kernel<<<grid, kThreads, Layout::kAlloc,
                                        static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, p);
     g_last_launches = 1;
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;

@@ -40,8 +40,8 @@
 // block 1), passed on through a "turn" mbarrier, so one warpgroup's loads,
 // row max and waits overlap the other's exponentials instead of both
 // warpgroups doing the same phase at the same time.
-// Shared memory: Q0, Q1, P0, P1 (32 KiB each), a ring of K_STAGES K tiles and
-// a ring of V_STAGES V tiles (32 KiB each), all in the 128-byte swizzle that
+// Shared memory: Q0, Q1, P0, P1 (32 KiB each), a ring of kKStages K tiles and
+// a ring of kVStages V tiles (32 KiB each), all in the 128-byte swizzle that
 // TMA writes and tcgen05 reads.  K and V have separate rings: K(j+1) is used
 // early in step j (right after the softmax frees S) and released soon after,
 // while V(j) is held until the end of step j's softmax, so V gets the
@@ -60,14 +60,10 @@ constexpr int kThreads = 384;
 constexpr int kMmaWarp0 = 8;   // issues query block 0's MMAs, allocates TMEM
 constexpr int kLoadWarp = 9;
 constexpr int kMmaWarp1 = 10;  // issues query block 1's MMAs
-// Exponentials of unmasked blocks: in every 16 column pairs of a 32-key
-// chunk, pairs with index below kPolyPairs go to the FMA-pipe polynomial,
-// the rest to the MUFU ex2 unit.  Measured slower than MUFU alone on B200,
-// so it is off unless SDPA10_POLY_PAIRS is set at build time.
-#ifndef SDPA10_POLY_PAIRS
-#define SDPA10_POLY_PAIRS 0
-#endif
-constexpr int kPolyPairs = SDPA10_POLY_PAIRS;
+// A warpgroup passes the exponential turn on after 12 of its 16 P chunks:
+// the next warpgroup's wake-up then overlaps the tail of the loop (measured
+// best among hand-off points 6..16 on B200).
+constexpr int kTurnChunk = 12;
 // Register split (per thread): launched at 65536 / 384 -> 168; the control
 // warpgroup (two MMA issuers, TMA, one idle warp) drops to 72 so each softmax
 // warpgroup can rise to 216: 2 * 128 * 216 + 128 * 72 = 384 * 168.
@@ -118,18 +114,17 @@ struct PairCursor {
 };
 
 // ------------------------------------------------------------------ layout
-constexpr int K_STAGES = 1;
-constexpr int V_STAGES = 2;
-template <int K_STAGES_>
+constexpr int kKStages = 1;  // K tiles in flight
+constexpr int kVStages = 2;  // V tiles in flight
 struct SmemLayout {
     static constexpr int kQ = 0;                              // Q0, Q1
     static constexpr int kP = 2 * kTileBytes;                 // P0, P1
     static constexpr int kK = 4 * kTileBytes;                 // K ring
-    static constexpr int kV = kK + K_STAGES * kTileBytes;     // V ring
-    static constexpr int kBars = kV + V_STAGES * kTileBytes;  // mbarriers
-    static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = 4 + K_STAGES,
-                         bVFull = 4 + 2 * K_STAGES, bVEmpty = bVFull + V_STAGES,
-                         bSFull = bVEmpty + V_STAGES,
+    static constexpr int kV = kK + kKStages * kTileBytes;     // V ring
+    static constexpr int kBars = kV + kVStages * kTileBytes;  // mbarriers
+    static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = 4 + kKStages,
+                         bVFull = 4 + 2 * kKStages, bVEmpty = bVFull + kVStages,
+                         bSFull = bVEmpty + kVStages,
                          bSFree = bSFull + 2, bPFull = bSFree + 2, bOFull = bPFull + 2,
                          bOEmpty = bOFull + 2, bTurn = bOEmpty + 2, bDrain = bTurn + 1,
                          kNumBars = bDrain + 2;
@@ -139,43 +134,52 @@ struct SmemLayout {
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
 
-// ------------------------------------------------------------------ exp2 on the FMA pipe
-// 2^x for a pair of FP32 values without the MUFU unit (Cody-Waite style range
-// reduction): x = k + f with k = round(x) and f in [-1/2, 1/2]; 2^f by a
-// degree-3 polynomial whose coefficients are a Remez (minimax relative
-// error) fit of 2^f on [-1/2, 1/2], max relative error 7.5e-5 in FP32 --
-// far below the BF16 rounding P gets next; 2^k enters by adding k to the
-// exponent field.  k comes from adding 1.5 * 2^23, which leaves round(x) in
-// the low mantissa bits.  Inputs below -125 are clamped there (2^-125 ~
-// 2.4e-38 stays a normal number); only unmasked blocks use this path.
-__device__ __forceinline__ uint64_t exp2_poly_x2(uint64_t x2) {
-    constexpr float kRound = 12582912.0f;  // 1.5 * 2^23
-    constexpr float c0 = 0.99992805719375610f, c1 = 0.69326096773147583f,
-                    c2 = 0.24261112511157990f, c3 = 0.05517166852951050f;
-    float x0, x1;
-    ptx::f2_unpack(x2, x0, x1);
-    const uint64_t x = ptx::f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
-    const uint64_t t = ptx::f2_add(x, ptx::f2_pack(kRound, kRound));     // 1.5*2^23 + k
-    const uint64_t kf = ptx::f2_add(t, ptx::f2_pack(-kRound, -kRound));  // k
-    const uint64_t f = ptx::f2_fma(kf, ptx::f2_pack(-1.f, -1.f), x);     // x - k
-    uint64_t p = ptx::f2_fma(ptx::f2_pack(c3, c3), f, ptx::f2_pack(c2, c2));
-    p = ptx::f2_fma(p, f, ptx::f2_pack(c1, c1));
-    p = ptx::f2_fma(p, f, ptx::f2_pack(c0, c0));
-    float t0, t1, p0, p1;
-    ptx::f2_unpack(t, t0, t1);
-    ptx::f2_unpack(p, p0, p1);
-    const float r0 = __int_as_float(__float_as_int(p0) + (__float_as_int(t0) << 23));
-    const float r1 = __int_as_float(__float_as_int(p1) + (__float_as_int(t1) << 23));
-    return ptx::f2_pack(r0, r1);
+// ------------------------------------------------------------------ exponentials
+// P = 2^(s c - m c) for one 128-key row on the MUFU ex2 unit: FP32 row sum
+// returned in two accumulators, BF16 P written to this row of the
+// shared-memory P tile (16-byte chunk cc at row_base + (cc / 8) * 16 KiB +
+// ((cc % 8) ^ xor) * 16).  When `pass_turn` is set the warp arrives on the
+// turn barrier after kTurnChunk chunks.
+__device__ __forceinline__ void exp_row(const float (&s)[128], float c2, float nmc,
+                                        uint32_t p_row, uint32_t p_xor, float& sum_a,
+                                        float& sum_b, bool pass_turn, uint32_t turn, int lane) {
+    const uint64_t c2x2 = ptx::f2_pack(c2, c2), nmc2 = ptx::f2_pack(nmc, nmc);
+    uint64_t sum2a = ptx::f2_pack(0.f, 0.f), sum2b = sum2a;
+#pragma unroll
+    for (int cc = 0; cc < 16; ++cc) {
+        uint32_t w[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int e0 = 8 * cc + 2 * k;
+            const uint64_t x = ptx::f2_fma(ptx::f2_pack(s[e0], s[e0 + 1]), c2x2, nmc2);
+            float x0, x1;
+            ptx::f2_unpack(x, x0, x1);
+            const float p0 = ptx::ex2(x0), p1 = ptx::ex2(x1);
+            const uint64_t e = ptx::f2_pack(p0, p1);
+            if (k & 1) sum2b = ptx::f2_add(sum2b, e);
+            else sum2a = ptx::f2_add(sum2a, e);
+            w[k] = ptx::pack_bf16x2(p0, p1);
+        }
+        ptx::st_shared_v4(p_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ p_xor) << 4), w[0],
+                          w[1], w[2], w[3]);
+        if (cc == kTurnChunk - 1 && pass_turn) {
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(turn);
+        }
+    }
+    float a0, a1, b0, b1;
+    ptx::f2_unpack(sum2a, a0, a1);
+    ptx::f2_unpack(sum2b, b0, b1);
+    sum_a += a0 + a1;
+    sum_b += b0 + b1;
 }
 
 // ------------------------------------------------------------------ softmax
 // One softmax warpgroup: thread r owns query row r of its block (TMEM lane r).
-template <int K_STAGES>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& wc,
                                              uint32_t tmem, uint32_t sP, uint32_t bars, int wg,
                                              int warp_in_wg, int lane) {
-    using L = SmemLayout<K_STAGES>;
+    using L = SmemLayout;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
     const int r = warp_in_wg * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(warp_in_wg * 32) << 16;
@@ -190,17 +194,22 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
     const uint32_t p_row = sP + wg * kTileBytes + (r >> 3) * 1024 + (r & 7) * 128;
     const uint32_t p_xor = static_cast<uint32_t>(r & 7);
     const float c2 = p.scale_log2;
-    const uint64_t c2x2 = ptx::f2_pack(c2, c2);
 
     const uint32_t b_turn = bar(L::bTurn);
-    uint32_t cnt = 0;   // S blocks this warpgroup has processed (all pairs)
-    uint32_t seq0 = 0;  // exponential phases of both warpgroups before this pair
+    // Exponential turns strictly alternate: at key block j < min(n0, n1) of
+    // a pair, block 0 takes turn 2K and block 1 turn 2K + 1 (K counts such
+    // rounds over all pairs); a block's key blocks past that run without a
+    // turn.  Each wait then finds the turn barrier at most one phase short,
+    // which its single parity bit can tell apart.
+    uint32_t cnt = 0;     // S blocks this warpgroup has processed (all pairs)
+    uint32_t rounds = 0;  // alternation rounds before this pair
     PairCursor c;
     c.start(p);
     for (; c.valid(p); c.next(p)) {
         const int n = c.n[wg];
-        const uint32_t seq = seq0;
-        seq0 += static_cast<uint32_t>(c.n[0] + c.n[1]);
+        const int n_turns = min(c.n[0], c.n[1]);
+        const uint32_t round0 = rounds;
+        rounds += static_cast<uint32_t>(n_turns);
         if (n == 0) continue;
         const int qb = c.qb0 + wg;
         const int row = qb * kBlockM + r;
@@ -259,7 +268,6 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
             }
             const float m_ref = (m_run == -CUDART_INF_F) ? 0.f : m_run;
             const float neg_mc = -m_ref * c2;
-            const uint64_t nmc2 = ptx::f2_pack(neg_mc, neg_mc);
 
             // The previous P V of this block must be done before its P
             // buffer is rewritten (and before O is rescaled).
@@ -289,48 +297,17 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
                 ptx::tc_fence_before();
             }
 
-            // Our turn on the exponential unit: phase index m in the global
-            // order (block 0 before block 1 at each key block j).
-            const uint32_t m = wg == 0 ? seq + j + min(j, c.n[1])
-                                       : seq + min(j + 1, c.n[0]) + j;
-            if (m > 0 && !wait_bar_warp(b_turn, (m - 1) & 1, wc)) return;
-            // P = 2^(s c - m c), 8 keys -> one 16-byte chunk of the P row.
-            uint64_t sum2a = ptx::f2_pack(0.f, 0.f), sum2b = sum2a;
-#pragma unroll
-            for (int cc = 0; cc < 16; ++cc) {
-                uint32_t w[4];
-#pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int e0 = 8 * cc + 2 * k;
-                    const uint64_t x = ptx::f2_fma(ptx::f2_pack(s[e0], s[e0 + 1]), c2x2, nmc2);
-                    uint64_t e;
-                    if (kPolyPairs > 0 && !masked && ((cc * 4 + k) & 15) < kPolyPairs) {
-                        e = exp2_poly_x2(x);
-                    } else {
-                        float x0, x1;
-                        ptx::f2_unpack(x, x0, x1);
-                        e = ptx::f2_pack(ptx::ex2(x0), ptx::ex2(x1));
-                    }
-                    if (k & 1) sum2b = ptx::f2_add(sum2b, e);
-                    else sum2a = ptx::f2_add(sum2a, e);
-                    w[k] = ptx::pack_bf16x2_from(e);
-                }
-                ptx::st_shared_v4(p_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ p_xor) << 4),
-                                  w[0], w[1], w[2], w[3]);
-            }
-            // The exponentials are done: pass the turn on first, then make P
-            // visible to the tensor core (async proxy) and hand it over.
-            __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(b_turn);
+            // Our turn on the exponential unit: wait for turn m - 1.
+            const bool turn = j < n_turns;
+            const uint32_t m = 2 * (round0 + j) + wg;
+            if (turn && m > 0 && !wait_bar_warp(b_turn, (m - 1) & 1, wc)) return;
+            float sum_a = 0.f, sum_b = 0.f;
+            exp_row(s, c2, neg_mc, p_row, p_xor, sum_a, sum_b, turn, b_turn, lane);
+            // Make P visible to the tensor core (async proxy) and hand it over.
             ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(b_pfull);
-            {
-                float a0, a1, b0, b1;
-                ptx::f2_unpack(sum2a, a0, a1);
-                ptx::f2_unpack(sum2b, b0, b1);
-                l_run = l_run * alpha + ((a0 + a1) + (b0 + b1));
-            }
+            l_run = l_run * alpha + (sum_a + sum_b);
 
             if (j == n - 1) {
                 // Epilogue: O / l -> BF16 rows, LSE in natural log.
@@ -375,13 +352,12 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
 }
 
 // ------------------------------------------------------------------ kernel
-template <int K_STAGES>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ FwdParams p) {
-    using L = SmemLayout<K_STAGES>;
+    using L = SmemLayout;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -408,11 +384,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(bar(L::bOFull + i), 1);
             ptx::mbar_init(bar(L::bOEmpty + i), 4);
         }
-        for (int i = 0; i < K_STAGES; ++i) {
+        for (int i = 0; i < kKStages; ++i) {
             ptx::mbar_init(bar(L::bKFull + i), 1);
             ptx::mbar_init(bar(L::bKEmpty + i), 2);  // one arrival per MMA issuer
         }
-        for (int i = 0; i < V_STAGES; ++i) {
+        for (int i = 0; i < kVStages; ++i) {
             ptx::mbar_init(bar(L::bVFull + i), 1);
             ptx::mbar_init(bar(L::bVEmpty + i), 2);
         }
@@ -453,16 +429,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tma_load_4d(dst + kHalfTileBytes, tm, full, 64, c.g, j * kBlockN, c.b, pol_kv);
             };
             auto load_k = [&](const PairCursor& c, int j) -> bool {
-                const int slot = k_loads % K_STAGES;
-                if (!wait_bar(bar(L::bKEmpty + slot), ((k_loads / K_STAGES) & 1) ^ 1, wc))
+                const int slot = k_loads % kKStages;
+                if (!wait_bar(bar(L::bKEmpty + slot), ((k_loads / kKStages) & 1) ^ 1, wc))
                     return false;
                 load_tile(&tm_k, sK + slot * kTileBytes, bar(L::bKFull + slot), c, j);
                 ++k_loads;
                 return true;
             };
             auto load_v = [&](const PairCursor& c, int j) -> bool {
-                const int slot = v_loads % V_STAGES;
-                if (!wait_bar(bar(L::bVEmpty + slot), ((v_loads / V_STAGES) & 1) ^ 1, wc))
+                const int slot = v_loads % kVStages;
+                if (!wait_bar(bar(L::bVEmpty + slot), ((v_loads / kVStages) & 1) ^ 1, wc))
                     return false;
                 load_tile(&tm_v, sV + slot * kTileBytes, bar(L::bVFull + slot), c, j);
                 ++v_loads;
@@ -496,13 +472,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             // Drain: every issued copy must land before the CTA may exit.
-            for (int i = 0; i < K_STAGES && i < static_cast<int>(k_loads); ++i) {
+            for (int i = 0; i < kKStages && i < static_cast<int>(k_loads); ++i) {
                 const uint32_t f = k_loads - 1 - i;
-                wait_slow(bar(L::bKFull + f % K_STAGES), (f / K_STAGES) & 1, wc, false);
+                wait_slow(bar(L::bKFull + f % kKStages), (f / kKStages) & 1, wc, false);
             }
-            for (int i = 0; i < V_STAGES && i < static_cast<int>(v_loads); ++i) {
+            for (int i = 0; i < kVStages && i < static_cast<int>(v_loads); ++i) {
                 const uint32_t f = v_loads - 1 - i;
-                wait_slow(bar(L::bVFull + f % V_STAGES), (f / V_STAGES) & 1, wc, false);
+                wait_slow(bar(L::bVFull + f % kVStages), (f / kVStages) & 1, wc, false);
             }
 #pragma unroll
             for (int i = 0; i < 2; ++i)
@@ -528,22 +504,22 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t v_lo = desc_lo_sw128(sV, kHalfTileBytes);
             const uint32_t s_tm = tmem + i * 128, o_tm = tmem + 256 + i * 128;
             auto wait_k = [&]() -> bool {
-                return wait_bar(bar(L::bKFull + k_used % K_STAGES), (k_used / K_STAGES) & 1, wc);
+                return wait_bar(bar(L::bKFull + k_used % kKStages), (k_used / kKStages) & 1, wc);
             };
             auto wait_v = [&]() -> bool {
-                return wait_bar(bar(L::bVFull + v_used % V_STAGES), (v_used / V_STAGES) & 1, wc);
+                return wait_bar(bar(L::bVFull + v_used % kVStages), (v_used / kVStages) & 1, wc);
             };
             // A tile this block does not use: once it has landed (so the slot's
             // previous use is released), give up this issuer's share of it.
             auto skip_k = [&]() -> bool {
                 if (!wait_k()) return false;
-                ptx::mbar_arrive(bar(L::bKEmpty + k_used % K_STAGES));
+                ptx::mbar_arrive(bar(L::bKEmpty + k_used % kKStages));
                 ++k_used;
                 return true;
             };
             auto skip_v = [&]() -> bool {
                 if (!wait_v()) return false;
-                ptx::mbar_arrive(bar(L::bVEmpty + v_used % V_STAGES));
+                ptx::mbar_arrive(bar(L::bVEmpty + v_used % kVStages));
                 ++v_used;
                 return true;
             };
@@ -552,7 +528,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_k()) return false;
                 if (s_cnt > 0 && !wait_bar(bar(L::bSFree + i), (s_cnt - 1) & 1, wc)) return false;
                 ptx::tc_fence_after();
-                const uint32_t ka = k_lo + (((k_used % K_STAGES) * kTileBytes) >> 4);
+                const uint32_t ka = k_lo + (((k_used % kKStages) * kTileBytes) >> 4);
 #pragma unroll
                 for (int k = 0; k < kHeadDim / 16; ++k) {
                     // K-major, 128-byte swizzle: 16 BF16 (32 bytes) per step
@@ -563,7 +539,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::mma_commit(bar(L::bSFull + i));
                 if (last_of_pair) ptx::mma_commit(bar(L::bQEmpty + i));
-                ptx::mma_commit(bar(L::bKEmpty + k_used % K_STAGES));
+                ptx::mma_commit(bar(L::bKEmpty + k_used % kKStages));
                 ++k_used;
                 ++s_cnt;
                 return true;
@@ -573,7 +549,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_v()) return false;
                 if (!wait_bar(bar(L::bPFull + i), pv_cnt & 1, wc)) return false;
                 ptx::tc_fence_after();
-                const uint32_t va = v_lo + (((v_used % V_STAGES) * kTileBytes) >> 4);
+                const uint32_t va = v_lo + (((v_used % kVStages) * kTileBytes) >> 4);
 #pragma unroll
                 for (int k = 0; k < kBlockN / 16; ++k) {
                     // A = P (K-major like Q); B = V, MN-major (head dim
@@ -585,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 (acc || k > 0) ? 1u : 0u);
                 }
                 ptx::mma_commit(bar(L::bOFull + i));
-                ptx::mma_commit(bar(L::bVEmpty + v_used % V_STAGES));
+                ptx::mma_commit(bar(L::bVEmpty + v_used % kVStages));
                 ++v_used;
                 ++pv_cnt;
                 return true;
@@ -625,7 +601,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp < 8) {
         ptx::reg_alloc<kRegsSoftmax>();
-        softmax_role<K_STAGES>(p, wc, tmem, sP, bars, warp >> 2, warp & 3, lane);
+        softmax_role(p, wc, tmem, sP, bars, warp >> 2, warp & 3, lane);
     } else {
         ptx::reg_dealloc<kRegsControl>();  // idle warps of the control warpgroup
     }

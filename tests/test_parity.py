@@ -99,6 +99,29 @@ def test_deterministic():
     assert torch.equal(o1, o2) and torch.equal(l1, l2)
 
 
+@pytest.mark.parametrize("s", [4096, 3968, 1152])
+def test_causal_turn_order_many_launches(s):
+    # In a causal pair the second query block has one key block more than
+    # the first, and an odd block count leaves the last pair's second block
+    # empty.  The two softmax warpgroups' turn order on the exponential unit
+    # must survive both over many launches: a lost turn ends in the bounded
+    # wait's timeout status, and every launch must give the same bits.
+    b, h = 2, 16
+    q, k, v = make_qkv(b, h, h, s, s, seed=6450 + s)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o0, l0 = run_gpu(q, k, v, True, SCALE)
+    o, lse = torch.empty_like(o0), torch.empty_like(l0)
+    for i in range(200):
+        attn.attn_fwd(qd, kd, vd, causal=True, scale=SCALE, o=o, lse=lse)
+        if i % 50 == 49:
+            assert attn.attn_status() == attn.ATTN_OK, f"launch {i}"
+            assert torch.equal(o, o0) and torch.equal(lse, l0), f"launch {i}"
+    rows = sample_rows(b, h, s, 64, seed=6460 + s)
+    o_ref, l_ref, _ = oracle.attn_fwd(q, k, v, True, SCALE, rows=rows)
+    oo, ll = gather_rows(o0, l0, rows)
+    assert_within(metrics(oo, ll, o_ref, l_ref), f"causal s={s}")
+
+
 def test_outputs_stay_in_bounds():
     # o and lse sit inside larger buffers; the guard regions must be untouched.
     b, h, s = 1, 2, 200
