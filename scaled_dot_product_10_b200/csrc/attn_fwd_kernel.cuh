@@ -140,10 +140,9 @@ struct SmemLayout {
 // shared-memory P tile (16-byte chunk cc at row_base + (cc / 8) * 16 KiB +
 // ((cc % 8) ^ xor) * 16).  When `pass_turn` is set the warp arrives on the
 // turn barrier after kTurnChunk chunks.
-__device__ __forceinline__ void exp_row(const float (&s)[128], float c2, float nmc,
+__device__ __forceinline__ void exp_row(const float (&s)[128], uint64_t c2x2, uint64_t nmc2,
                                         uint32_t p_row, uint32_t p_xor, float& sum_a,
                                         float& sum_b, bool pass_turn, uint32_t turn, int lane) {
-    const uint64_t c2x2 = ptx::f2_pack(c2, c2), nmc2 = ptx::f2_pack(nmc, nmc);
     uint64_t sum2a = ptx::f2_pack(0.f, 0.f), sum2b = sum2a;
 #pragma unroll
     for (int cc = 0; cc < 16; ++cc) {
@@ -194,6 +193,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
     const uint32_t p_row = sP + wg * kTileBytes + (r >> 3) * 1024 + (r & 7) * 128;
     const uint32_t p_xor = static_cast<uint32_t>(r & 7);
     const float c2 = p.scale_log2;
+    const uint64_t c2x2 = ptx::f2_pack(c2, c2);
 
     const uint32_t b_turn = bar(L::bTurn);
     // Exponential turns strictly alternate: at key block j < min(n0, n1) of
@@ -302,7 +302,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
             const uint32_t m = 2 * (round0 + j) + wg;
             if (turn && m > 0 && !wait_bar_warp(b_turn, (m - 1) & 1, wc)) return;
             float sum_a = 0.f, sum_b = 0.f;
-            exp_row(s, c2, neg_mc, p_row, p_xor, sum_a, sum_b, turn, b_turn, lane);
+            exp_row(s, c2x2, ptx::f2_pack(neg_mc, neg_mc), p_row, p_xor, sum_a, sum_b, turn, b_turn,
+                    lane);
             // Make P visible to the tensor core (async proxy) and hand it over.
             ptx::fence_proxy_async_smem();
             __syncwarp();
