@@ -128,6 +128,92 @@ int attn_fwd_host_static(const void* q, const void* k, const void* v, void* o, f
                          int causal, float scale, void* stream);
 
 /*
+ * Split-KV forward (split the key sequence into ranges, then merge).
+ *
+ * The same result as attn_fwd, computed as one work item per (query-block
+ * pair, key range) and then merged: for a key set split into ranges r, with
+ * O_r the softmax-weighted average of V over range r and LSE_r the
+ * log-sum-exp of that range's scaled scores,
+ *     LSE = log sum_r exp(LSE_r),    O = sum_r exp(LSE_r - LSE) O_r
+ * (the rkmt.cn GPU attention operator page's "local attention, then global
+ * reduction", section 3.1.1, applied to whole key ranges).  It pays off when
+ * batch * h_q * ceil(s_q / 256) work items leave most SMs idle, e.g. few
+ * query rows over a long key sequence.
+ *
+ * attn_fwd_num_splits -- the key-range count this library would pick on the
+ * current device: 1 when the pairs already fill the SMs, else about
+ * #SMs / pairs, at most ceil(s_k / 128).  0 on invalid sizes.
+ */
+int attn_fwd_num_splits(int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal);
+
+/* Device workspace bytes attn_fwd_split needs for num_splits ranges
+ * (num_splits * batch * h_q * s_q * (128 + 1) FP32 values, rounded; 0 on bad
+ * sizes). */
+size_t attn_fwd_split_workspace_bytes(int batch, int h_q, int s_q, int num_splits);
+
+/*
+ * attn_fwd_split -- attn_fwd through num_splits key ranges (>= 1; more than
+ * ceil(s_k / 128) is reduced to that, and the ranges are ceil(n_kb / n)
+ * key blocks of 128 each, the last one shorter).  Arguments, layouts and
+ * errors as attn_fwd, plus:
+ *
+ *   workspace  device buffer of at least
+ *              attn_fwd_split_workspace_bytes(batch, h_q, s_q, num_splits)
+ *              bytes, 256-byte aligned, owned by the caller (per-range
+ *              partials: FP32 O_r [n][batch][h_q][s_q][128], then FP32 LSE_r
+ *              [n][batch][h_q][s_q]); ATTN_ERR_INVALID if smaller or null,
+ *              ATTN_ERR_ALIGN if misaligned.
+ *
+ * Two launches on `stream` (the forward writing partials, then the merge);
+ * asynchronous; allocates nothing.  Results agree with attn_fwd within
+ * rounding (bit for bit when num_splits is 1).
+ */
+int attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal,
+                   float scale, int num_splits, void* workspace, size_t workspace_bytes,
+                   void* stream);
+
+/*
+ * attn_fwd_partials -- the partial of one key range: the forward over the
+ * keys given, written unmerged for attn_merge_partials.  What a rank of a
+ * key-sequence (context-parallel) split computes on its own key shard before
+ * the partials are gathered.  Arguments and errors as attn_fwd, except:
+ *
+ *   o_part    device, fp32 [batch, h_q, s_q, d] (written): softmax over these
+ *             keys times V, already divided by the range's row sum; 16-byte
+ *             aligned
+ *   lse_part  device, fp32 [batch, h_q, s_q] (written): natural-log
+ *             log-sum-exp of the range's scaled scores
+ *
+ * One launch; asynchronous; allocates nothing.
+ */
+int attn_fwd_partials(const void* q, const void* k, const void* v, float* o_part,
+                      float* lse_part, int batch, int h_q, int h_kv, int s_q, int s_k, int d,
+                      int causal, float scale, void* stream);
+
+/*
+ * attn_merge_partials -- the merge step alone, for partials computed
+ * elsewhere (for example over key ranges held by different GPUs and gathered
+ * onto this one):
+ *
+ *   o_parts    device, fp32 [n_parts, batch, h_q, s_q, d], each part already
+ *              normalised over its own keys (16-byte aligned)
+ *   lse_parts  device, fp32 [n_parts, batch, h_q, s_q], natural log; a part
+ *              with no keys for a row carries -inf there (weight 0; its O
+ *              values for that row are not read)
+ *   o          device, bf16 [batch, s_q, h_q, d] (written, 16-byte aligned)
+ *   lse        device, fp32 [batch, h_q, s_q] (written)
+ *   d          must be 128
+ *
+ * A row whose parts are all -inf gets O = 0 and LSE = -inf.  One launch on
+ * `stream`; asynchronous; allocates nothing.  ATTN_ERR_INVALID on a null
+ * pointer or a count <= 0, ATTN_ERR_UNSUPPORTED if d != 128, ATTN_ERR_ALIGN
+ * on misaligned buffers.
+ */
+int attn_merge_partials(const float* o_parts, const float* lse_parts, int n_parts, int batch,
+                        int h_q, int s_q, int d, void* o, float* lse, void* stream);
+
+/*
  * attn_status -- synchronise `stream`, then read and clear the calling
  * device's kernel status word.  Returns ATTN_OK, ATTN_ERR_TIMEOUT if a kernel
  * launched since the last call gave up a bounded wait, or ATTN_ERR_CUDA if
@@ -153,7 +239,8 @@ int attn_set_wait_timeout_ns(uint64_t ns);
  */
 int attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
 
-/* Number of kernel launches the last attn_fwd / attn_fwd_host made (1). */
+/* Number of kernel launches the last forward call made (1; 2 for
+ * attn_fwd_split: forward + merge). */
 int attn_last_launch_count(void);
 
 #ifdef __cplusplus

@@ -33,6 +33,13 @@ _SIGNATURES = [
     ("attn_fwd_host_workspace_bytes", ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
     ("attn_fwd_host_static", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
                                   _P]),
+    ("attn_fwd_num_splits", _I, [_I, _I, _I, _I, _I, _I, _I]),
+    ("attn_fwd_split_workspace_bytes", ctypes.c_size_t, [_I, _I, _I, _I]),
+    ("attn_fwd_split", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I,
+                            _P, ctypes.c_size_t, _P]),
+    ("attn_merge_partials", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
+    ("attn_fwd_partials", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
+                               _P]),
     ("attn_status", _I, [_P]),
     ("attn_strerror", ctypes.c_char_p, [_I]),
     ("attn_set_wait_timeout_ns", _I, [ctypes.c_uint64]),
@@ -122,6 +129,97 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, 
                                  float(scale), _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd")
+    return o, lse
+
+
+def num_splits(b, h_q, h_kv, s_q, s_k, causal=False, d=128) -> int:
+    """Key-range count the library picks for these sizes on the current device."""
+    return int(load_library().attn_fwd_num_splits(b, h_q, h_kv, s_q, s_k, d, int(bool(causal))))
+
+
+def split_workspace_bytes(b, h_q, s_q, n_splits) -> int:
+    return int(load_library().attn_fwd_split_workspace_bytes(b, h_q, s_q, n_splits))
+
+
+def attn_fwd_split(q, k, v, causal: bool = False, scale: float | None = None,
+                   n_splits: int | None = None, o=None, lse=None, workspace=None, stream=None):
+    """attn_fwd through ``n_splits`` key ranges and a merge (two launches).
+    ``n_splits`` None: the library's choice (:func:`num_splits`).  The
+    partials go to ``workspace`` (a CUDA uint8 tensor of at least
+    :func:`split_workspace_bytes` bytes; allocated here if None)."""
+    import torch
+    b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if n_splits is None:
+        n_splits = max(1, num_splits(b, h_q, h_kv, s_q, s_k, causal, d))
+    if o is None:
+        o = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.empty(split_workspace_bytes(b, h_q, s_q, n_splits), dtype=torch.uint8,
+                                device=q.device)
+    rc = load_library().attn_fwd_split(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                       lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
+                                       int(bool(causal)), float(scale), int(n_splits),
+                                       workspace.data_ptr(),
+                                       workspace.numel() * workspace.element_size(),
+                                       _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_split")
+    return o, lse
+
+
+def attn_fwd_partials(q, k, v, causal: bool = False, scale: float | None = None, o_part=None,
+                      lse_part=None, stream=None):
+    """The unmerged partial of the keys given: O_r FP32 [b, h_q, s_q, 128]
+    (normalised over these keys) and LSE_r FP32 [b, h_q, s_q]."""
+    import torch
+    b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if o_part is None:
+        o_part = torch.empty((b, h_q, s_q, d), dtype=torch.float32, device=q.device)
+    if lse_part is None:
+        lse_part = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
+    rc = load_library().attn_fwd_partials(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                          o_part.data_ptr(), lse_part.data_ptr(), b, h_q, h_kv,
+                                          s_q, s_k, d, int(bool(causal)), float(scale),
+                                          _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_partials")
+    return o_part, lse_part
+
+
+def merge_partials(o_parts, lse_parts, o=None, lse=None, stream=None):
+    """Merge per-key-range partials: ``o_parts`` FP32 [n, b, h_q, s_q, 128]
+    (each normalised over its own keys), ``lse_parts`` FP32 [n, b, h_q, s_q]
+    -> O BF16 [b, s_q, h_q, 128], LSE FP32 [b, h_q, s_q]."""
+    import torch
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
+        raise TypeError("partials must be float32")
+    if o_parts.dim() != 5 or lse_parts.dim() != 4 or not o_parts.is_contiguous() \
+            or not lse_parts.is_contiguous():
+        raise ValueError("o_parts [n, b, h, s, d] and lse_parts [n, b, h, s], contiguous")
+    n, b, h_q, s_q, d = o_parts.shape
+    if tuple(lse_parts.shape) != (n, b, h_q, s_q):
+        raise ValueError("o_parts and lse_parts shapes disagree")
+    if o is None:
+        o = torch.empty((b, s_q, h_q, d), dtype=torch.bfloat16, device=o_parts.device)
+    if lse is None:
+        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=o_parts.device)
+    rc = load_library().attn_merge_partials(o_parts.data_ptr(), lse_parts.data_ptr(), n, b, h_q,
+                                            s_q, d, o.data_ptr(), lse.data_ptr(),
+                                            _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_merge_partials")
     return o, lse
 
 

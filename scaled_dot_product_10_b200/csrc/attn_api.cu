@@ -12,6 +12,7 @@
 
 #include "attn_fwd.h"
 #include "attn_fwd_kernel.cuh"
+#include "attn_merge.cuh"
 
 namespace {
 
@@ -115,17 +116,30 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
 
 size_t round_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
-}  // namespace
+// Effective key ranges for a requested count: ceil(n_kb / n) key blocks per
+// range, and as many ranges as that takes.
+void split_shape(int s_k, int num_splits, int* n_splits, int* kb_per_split) {
+    const int n_kb = (s_k + kBlockN - 1) / kBlockN;
+    const int n = num_splits < 1 ? 1 : (num_splits > n_kb ? n_kb : num_splits);
+    *kb_per_split = (n_kb + n - 1) / n;
+    *n_splits = (n_kb + *kb_per_split - 1) / *kb_per_split;
+}
 
-extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
-                        int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal,
-                        float scale, void* stream) {
-    int rc = validate(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale);
-    if (rc != ATTN_OK) return rc;
+size_t split_workspace_bytes(int batch, int h_q, int s_q, int n_splits) {
+    const size_t rows = static_cast<size_t>(batch) * h_q * s_q;
+    return round_up(static_cast<size_t>(n_splits) * rows * kHeadDim * 4, 256) +
+           static_cast<size_t>(n_splits) * rows * 4;
+}
+
+// The forward launch shared by attn_fwd and attn_fwd_split (arguments
+// already validated).  o_part / lse_part null: O and LSE directly.
+int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int batch,
+               int h_q, int h_kv, int s_q, int s_k, int causal, float scale, int n_splits,
+               int kb_per_split, float* o_part, float* lse_part, void* stream) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
     DeviceState* st = nullptr;
-    rc = init_device(dev, &st);
+    const int rc = init_device(dev, &st);
     if (rc != ATTN_OK) return rc;
 
     CUtensorMap tq, tk, tv;
@@ -144,7 +158,9 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
     p.n_kb = (s_k + kBlockN - 1) / kBlockN;
     p.causal = causal;
     p.n_pairs = (p.n_qb + 1) / 2;
-    p.num_tiles = batch * h_q * p.n_pairs;
+    p.n_splits = n_splits;
+    p.kb_per_split = kb_per_split;
+    p.num_tiles = batch * h_q * p.n_pairs * n_splits;
     const size_t unit_bytes = 2ull * s_k * kHeadDim * 2;  // K and V of one (batch, kv head)
     const size_t per_sec = kL2SectionBytes / (unit_bytes ? unit_bytes : 1);
     const int units_total = batch * h_kv;
@@ -152,6 +168,8 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
+    p.o_part = o_part;
+    p.lse_part = lse_part;
     p.timeout_ns = g_timeout_ns;
     p.status = st->status;
 
@@ -161,6 +179,126 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
     g_last_launches = 1;
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     return ATTN_OK;
+}
+
+int launch_merge(const float* o_part, const float* lse_part, int n_parts, int batch, int h_q,
+                 int s_q, int keys_per_part, int s_k, int causal, void* o, float* lse,
+                 void* stream) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    DeviceState* st = nullptr;
+    const int rc = init_device(dev, &st);
+    if (rc != ATTN_OK) return rc;
+    MergeParams m{};
+    m.o_part = o_part;
+    m.lse_part = lse_part;
+    m.n_parts = n_parts;
+    m.batch = batch;
+    m.h_q = h_q;
+    m.s_q = s_q;
+    m.keys_per_part = keys_per_part;
+    m.s_k = s_k;
+    m.causal = causal;
+    m.o = static_cast<__nv_bfloat16*>(o);
+    m.lse = lse;
+    const size_t rows = static_cast<size_t>(batch) * h_q * s_q;
+    const size_t per_block = kMergeThreads / 32;
+    size_t blocks = (rows + per_block - 1) / per_block;
+    const size_t cap = static_cast<size_t>(st->num_sms) * 8;
+    if (blocks > cap) blocks = cap;
+    attn_merge_kernel<<<static_cast<unsigned>(blocks), kMergeThreads, 0,
+                        static_cast<cudaStream_t>(stream)>>>(m);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    return ATTN_OK;
+}
+
+}  // namespace
+
+extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal,
+                        float scale, void* stream) {
+    const int rc = validate(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale);
+    if (rc != ATTN_OK) return rc;
+    const int n_kb = (s_k + kBlockN - 1) / kBlockN;
+    return launch_fwd(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, causal, scale, 1, n_kb,
+                      nullptr, nullptr, stream);
+}
+
+extern "C" int attn_fwd_num_splits(int batch, int h_q, int h_kv, int s_q, int s_k, int d,
+                                   int causal) {
+    if (validate_sizes(batch, h_q, h_kv, s_q, s_k, d) != ATTN_OK) return 0;
+    if (causal != 0 && causal != 1) return 0;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    DeviceState* st = nullptr;
+    if (init_device(dev, &st) != ATTN_OK) return 0;
+    const long long pairs = static_cast<long long>(batch) * h_q * ((s_q + 2 * kBlockM - 1) / (2 * kBlockM));
+    const int n_kb = (s_k + kBlockN - 1) / kBlockN;
+    if (pairs >= st->num_sms) return 1;
+    long long n = st->num_sms / pairs;
+    if (n > n_kb) n = n_kb;
+    int n_splits = 1, kb = 1;
+    split_shape(s_k, static_cast<int>(n < 1 ? 1 : n), &n_splits, &kb);
+    return n_splits;
+}
+
+extern "C" size_t attn_fwd_split_workspace_bytes(int batch, int h_q, int s_q, int num_splits) {
+    if (batch <= 0 || h_q <= 0 || s_q <= 0 || num_splits <= 0) return 0;
+    return split_workspace_bytes(batch, h_q, s_q, num_splits);
+}
+
+extern "C" int attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* lse,
+                              int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal,
+                              float scale, int num_splits, void* workspace,
+                              size_t workspace_bytes, void* stream) {
+    int rc = validate(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale);
+    if (rc != ATTN_OK) return rc;
+    if (num_splits < 1 || !workspace) return ATTN_ERR_INVALID;
+    if (!aligned(workspace, 256)) return ATTN_ERR_ALIGN;
+    int n_splits = 1, kb_per_split = 1;
+    split_shape(s_k, num_splits, &n_splits, &kb_per_split);
+    const long long n_qb = (s_q + kBlockM - 1) / kBlockM;
+    if (static_cast<long long>(batch) * h_q * ((n_qb + 1) / 2) * n_splits > 0x7fffffffLL)
+        return ATTN_ERR_INVALID;
+    if (workspace_bytes < split_workspace_bytes(batch, h_q, s_q, n_splits)) return ATTN_ERR_INVALID;
+    const size_t rows = static_cast<size_t>(batch) * h_q * s_q;
+    float* o_part = static_cast<float*>(workspace);
+    float* lse_part = reinterpret_cast<float*>(static_cast<char*>(workspace) +
+                                               round_up(static_cast<size_t>(n_splits) * rows *
+                                                            kHeadDim * 4,
+                                                        256));
+    rc = launch_fwd(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, causal, scale, n_splits,
+                    kb_per_split, o_part, lse_part, stream);
+    if (rc != ATTN_OK) return rc;
+    rc = launch_merge(o_part, lse_part, n_splits, batch, h_q, s_q, kb_per_split * kBlockN, s_k,
+                      causal, o, lse, stream);
+    g_last_launches = 2;
+    return rc;
+}
+
+extern "C" int attn_fwd_partials(const void* q, const void* k, const void* v, float* o_part,
+                                 float* lse_part, int batch, int h_q, int h_kv, int s_q, int s_k,
+                                 int d, int causal, float scale, void* stream) {
+    const int rc = validate(q, k, v, o_part, lse_part, batch, h_q, h_kv, s_q, s_k, d, causal,
+                            scale);
+    if (rc != ATTN_OK) return rc;
+    const int n_kb = (s_k + kBlockN - 1) / kBlockN;
+    return launch_fwd(q, k, v, nullptr, nullptr, batch, h_q, h_kv, s_q, s_k, causal, scale, 1,
+                      n_kb, o_part, lse_part, stream);
+}
+
+extern "C" int attn_merge_partials(const float* o_parts, const float* lse_parts, int n_parts,
+                                   int batch, int h_q, int s_q, int d, void* o, float* lse,
+                                   void* stream) {
+    if (!o_parts || !lse_parts || !o || !lse) return ATTN_ERR_INVALID;
+    if (n_parts <= 0 || batch <= 0 || h_q <= 0 || s_q <= 0 || d <= 0) return ATTN_ERR_INVALID;
+    if (d != kHeadDim) return ATTN_ERR_UNSUPPORTED;
+    if (!aligned(o_parts, 16) || !aligned(o, 16) || !aligned(lse_parts, 4) || !aligned(lse, 4))
+        return ATTN_ERR_ALIGN;
+    const int rc = launch_merge(o_parts, lse_parts, n_parts, batch, h_q, s_q, 0, 0, 0, o, lse,
+                                stream);
+    g_last_launches = 1;
+    return rc;
 }
 
 extern "C" size_t attn_fwd_host_workspace_bytes(int batch, int h_q, int h_kv, int s_q, int s_k,

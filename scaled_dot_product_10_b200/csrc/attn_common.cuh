@@ -30,11 +30,18 @@ struct FwdParams {
     int n_kb;     // ceil(s_k / 128)
     int n_pairs;  // ceil(n_qb / 2): CTA tiles per (batch, head)
     int causal;
-    int num_tiles;
+    int num_tiles;          // work items: pairs x n_splits
     int units_per_section;  // (batch, kv head) units whose K/V share L2 at once
+    int n_splits;           // key ranges per pair (1: the whole key sequence)
+    int kb_per_split;       // key blocks per range
     float scale_log2;       // scale * log2(e)
     __nv_bfloat16* o;
     float* lse;
+    // Split-KV partials (null unless n_splits > 1 or a split launch): per key
+    // range r, O_r = softmax over that range times V, FP32
+    // [n_splits][batch][h_q][s_q][128], and LSE_r [n_splits][batch][h_q][s_q].
+    float* o_part;
+    float* lse_part;
     unsigned long long timeout_ns;
     unsigned int* status;
 };

@@ -71,22 +71,31 @@ constexpr uint32_t kRegsSoftmax = 216;
 constexpr uint32_t kRegsControl = 72;
 
 // ------------------------------------------------------------------ schedule
-// Pair index t -> (batch, query head, first query block).  Pairs are grouped
-// in sections of `units_per_section` (batch, kv head) units so the K/V of a
-// section stay resident in L2 while its pairs run; inside a section the order
-// is pair descending (longest causal work first), then unit, then the query
-// heads of the unit's group (adjacent heads share K/V).
+// Work item t -> (pair, key range): pair u = t / n_splits, key range
+// t % n_splits (the ranges of one pair are adjacent, so they share its Q
+// tiles in L2).  Pair u -> (batch, query head, first query block): pairs are
+// grouped in sections of `units_per_section` (batch, kv head) units so the
+// K/V of a section stay resident in L2 while its pairs run; inside a section
+// the order is pair descending (longest causal work first), then unit, then
+// the query heads of the unit's group (adjacent heads share K/V).  Items
+// whose key range no row of the pair may see (causal) are skipped by every
+// role alike.
 struct PairCursor {
     int t;
     int b, h, g, qb0;
-    int n[2];  // key/value blocks each query block of the pair visits (0: absent)
+    int split, kb0;  // key range of the item: key blocks kb0 .. kb0 + n[i] - 1
+    int n[2];        // key/value blocks each query block of the pair visits (0: none)
 
     __device__ __forceinline__ void decode(const FwdParams& p) {
+        const int u = t / p.n_splits;
+        split = t - u * p.n_splits;
+        kb0 = split * p.kb_per_split;
+        const int kb_end = min(p.n_kb, kb0 + p.kb_per_split);
         const int per_unit = p.group * p.n_pairs;
         const int units_total = p.batch * p.h_kv;
         const int G = p.units_per_section;
-        const int sec = t / (G * per_unit);
-        const int r = t - sec * G * per_unit;
+        const int sec = u / (G * per_unit);
+        const int r = u - sec * G * per_unit;
         const int Gs = min(G, units_total - sec * G);
         const int rank = r / (Gs * p.group);
         const int rem = r - rank * Gs * p.group;
@@ -98,16 +107,25 @@ struct PairCursor {
         h = g * p.group + h_local;
         qb0 = 2 * pair;
         // Causal (s_q == s_k): rows of block qb see key blocks 0..qb.
-        n[0] = p.causal ? min(p.n_kb, qb0 + 1) : p.n_kb;
-        n[1] = (qb0 + 1 < p.n_qb) ? (p.causal ? min(p.n_kb, qb0 + 2) : p.n_kb) : 0;
+        const int vis0 = p.causal ? min(kb_end, qb0 + 1) : kb_end;
+        const int vis1 = (qb0 + 1 < p.n_qb) ? (p.causal ? min(kb_end, qb0 + 2) : kb_end) : 0;
+        n[0] = max(0, vis0 - kb0);
+        n[1] = max(0, vis1 - kb0);
+    }
+    // Decode item t, moving on (by the grid stride) past items with no work.
+    __device__ __forceinline__ void settle(const FwdParams& p) {
+        for (; t < p.num_tiles; t += gridDim.x) {
+            decode(p);
+            if (n[0] > 0 || n[1] > 0) return;
+        }
     }
     __device__ __forceinline__ void start(const FwdParams& p) {
         t = blockIdx.x;
-        if (t < p.num_tiles) decode(p);
+        settle(p);
     }
     __device__ __forceinline__ void next(const FwdParams& p) {
         t += gridDim.x;
-        if (t < p.num_tiles) decode(p);
+        settle(p);
     }
     __device__ __forceinline__ bool valid(const FwdParams& p) const { return t < p.num_tiles; }
     __device__ __forceinline__ int iters() const { return max(n[0], n[1]); }
@@ -232,7 +250,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(b_sfree);
 
-            const int kv0 = j * kBlockN;
+            const int kv0 = (c.kb0 + j) * kBlockN;
             const bool diag = p.causal && (kv0 + kBlockN - 1 > qb * kBlockM);
             const bool masked = diag || kv0 + kBlockN > p.s_k;
             if (masked) {
@@ -311,41 +329,72 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
             l_run = l_run * alpha + (sum_a + sum_b);
 
             if (j == n - 1) {
-                // Epilogue: O / l -> BF16 rows, LSE in natural log.
+                // Epilogue: O / l -> BF16 rows (or FP32 partial rows of a key
+                // range), LSE in natural log.
                 if (!wait_bar_warp(b_ofull, cnt & 1, wc)) return;
                 ptx::tc_fence_after();
                 const float inv_l = 1.f / l_run;
                 const uint64_t il2 = ptx::f2_pack(inv_l, inv_l);
-                uint4* orow = reinterpret_cast<uint4*>(
-                    p.o + ((static_cast<size_t>(c.b) * p.s_q + row) * p.h_q + c.h) * kHeadDim);
+                const float lse_row = (m_ref * c2 + __log2f(l_run)) * 0.69314718055994531f;
+                const size_t row_id = (static_cast<size_t>(c.b) * p.h_q + c.h) * p.s_q + row;
+                if (p.o_part != nullptr) {
+                    const size_t part =
+                        static_cast<size_t>(c.split) * p.batch * p.h_q * p.s_q + row_id;
+                    float4* frow = reinterpret_cast<float4*>(p.o_part + part * kHeadDim);
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t ov[32];
-                    ptx::tmem_ld32(o_tmem + q * 32, ov);
-                    ptx::tmem_wait_ld();
-                    uint32_t w[16];
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t ov[32];
+                        ptx::tmem_ld32(o_tmem + q * 32, ov);
+                        ptx::tmem_wait_ld();
+                        if (row < p.s_q) {
 #pragma unroll
-                    for (int k = 0; k < 16; ++k) {
-                        const uint64_t v = ptx::f2_mul(
-                            ptx::f2_pack(__uint_as_float(ov[2 * k]), __uint_as_float(ov[2 * k + 1])),
-                            il2);
-                        float lo, hi;
-                        ptx::f2_unpack(v, lo, hi);
-                        w[k] = ptx::pack_bf16x2(lo, hi);
+                            for (int k = 0; k < 8; ++k) {
+                                float a0, a1, b0, b1;
+                                ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(__uint_as_float(ov[4 * k]),
+                                                                        __uint_as_float(ov[4 * k + 1])),
+                                                           il2),
+                                               a0, a1);
+                                ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(__uint_as_float(ov[4 * k + 2]),
+                                                                        __uint_as_float(ov[4 * k + 3])),
+                                                           il2),
+                                               b0, b1);
+                                frow[q * 8 + k] = make_float4(a0, a1, b0, b1);
+                            }
+                        }
                     }
-                    if (row < p.s_q) {
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(b_oempty);
+                    if (row < p.s_q) p.lse_part[part] = lse_row;
+                } else {
+                    uint4* orow = reinterpret_cast<uint4*>(
+                        p.o + ((static_cast<size_t>(c.b) * p.s_q + row) * p.h_q + c.h) * kHeadDim);
 #pragma unroll
-                        for (int k = 0; k < 4; ++k)
-                            orow[q * 4 + k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2],
-                                                         w[4 * k + 3]);
+                    for (int q = 0; q < 4; ++q) {
+                        uint32_t ov[32];
+                        ptx::tmem_ld32(o_tmem + q * 32, ov);
+                        ptx::tmem_wait_ld();
+                        uint32_t w[16];
+#pragma unroll
+                        for (int k = 0; k < 16; ++k) {
+                            const uint64_t v = ptx::f2_mul(
+                                ptx::f2_pack(__uint_as_float(ov[2 * k]), __uint_as_float(ov[2 * k + 1])),
+                                il2);
+                            float lo, hi;
+                            ptx::f2_unpack(v, lo, hi);
+                            w[k] = ptx::pack_bf16x2(lo, hi);
+                        }
+                        if (row < p.s_q) {
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                orow[q * 4 + k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2],
+                                                             w[4 * k + 3]);
+                        }
                     }
-                }
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(b_oempty);
-                if (row < p.s_q) {
-                    p.lse[(static_cast<size_t>(c.b) * p.h_q + c.h) * p.s_q + row] =
-                        (m_ref * c2 + __log2f(l_run)) * 0.69314718055994531f;
+                    ptx::tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(b_oempty);
+                    if (row < p.s_q) p.lse[row_id] = lse_row;
                 }
             }
         }
@@ -426,8 +475,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto load_tile = [&](const CUtensorMap* tm, uint32_t dst, uint32_t full, const PairCursor& c,
                                  int j) {
                 ptx::mbar_arrive_expect_tx(full, kTileBytes);
-                ptx::tma_load_4d(dst, tm, full, 0, c.g, j * kBlockN, c.b, pol_kv);
-                ptx::tma_load_4d(dst + kHalfTileBytes, tm, full, 64, c.g, j * kBlockN, c.b, pol_kv);
+                const int key0 = (c.kb0 + j) * kBlockN;
+                ptx::tma_load_4d(dst, tm, full, 0, c.g, key0, c.b, pol_kv);
+                ptx::tma_load_4d(dst + kHalfTileBytes, tm, full, 64, c.g, key0, c.b, pol_kv);
             };
             auto load_k = [&](const PairCursor& c, int j) -> bool {
                 const int slot = k_loads % kKStages;

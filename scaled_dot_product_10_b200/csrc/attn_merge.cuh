@@ -1,0 +1,82 @@
+// attn_merge.cuh -- combine per-key-range attention partials into O and LSE.
+//
+// Softmax over a key set split into ranges r: with O_r the softmax-weighted
+// average of V over range r and LSE_r the log-sum-exp of the range's scaled
+// scores, the whole set gives
+//     LSE = log sum_r exp(LSE_r)      O = sum_r exp(LSE_r - LSE) O_r,
+// the "local attention, then global reduction" merge of the rkmt.cn page
+// (section 3.1.1) applied to whole key ranges.  This is memory-bound work:
+// one warp per output row reads the row's partials (512 bytes each, 16 bytes
+// per lane) and writes 256 bytes of BF16 O and one FP32 LSE.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include <cstddef>
+
+namespace sdpa10 {
+
+struct MergeParams {
+    const float* o_part;    // [n_parts][rows][128] FP32, rows = batch * h_q * s_q
+    const float* lse_part;  // [n_parts][rows], natural log
+    int n_parts;
+    int batch, h_q, s_q;
+    // Key ranges of keys_per_part keys each, over s_k keys: range r holds
+    // keys [r * keys_per_part, (r + 1) * keys_per_part).  A range that holds
+    // no key of the row (past s_k, or past the row under the causal mask) is
+    // not read.  keys_per_part = 0: every part is read for every row (a part
+    // with LSE = -inf then carries no weight).
+    int keys_per_part, s_k, causal;
+    __nv_bfloat16* o;  // [batch][s_q][h_q][128]
+    float* lse;        // [batch][h_q][s_q]
+};
+
+constexpr int kMergeThreads = 256;
+
+__global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const MergeParams m) {
+    const int lane = threadIdx.x & 31;
+    const size_t rows = static_cast<size_t>(m.batch) * m.h_q * m.s_q;
+    const size_t warps = static_cast<size_t>(gridDim.x) * (kMergeThreads / 32);
+    for (size_t r = blockIdx.x * static_cast<size_t>(kMergeThreads / 32) + (threadIdx.x >> 5);
+         r < rows; r += warps) {
+        const int i = static_cast<int>(r % m.s_q);
+        const size_t bh = r / m.s_q;
+        const int h = static_cast<int>(bh % m.h_q);
+        const int b = static_cast<int>(bh / m.h_q);
+        int nv = m.n_parts;
+        if (m.keys_per_part > 0) {
+            nv = min(nv, (m.s_k + m.keys_per_part - 1) / m.keys_per_part);
+            if (m.causal) nv = min(nv, i / m.keys_per_part + 1);
+        }
+        float mx = -CUDART_INF_F;
+        for (int s = 0; s < nv; ++s) mx = fmaxf(mx, m.lse_part[static_cast<size_t>(s) * rows + r]);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        float wsum = 0.f;
+        if (mx != -CUDART_INF_F) {
+            for (int s = 0; s < nv; ++s) {
+                const size_t idx = static_cast<size_t>(s) * rows + r;
+                const float l_s = m.lse_part[idx];
+                if (l_s == -CUDART_INF_F) continue;  // no keys: its O is not read
+                const float w = expf(l_s - mx);
+                const float4 v = reinterpret_cast<const float4*>(m.o_part + idx * 128)[lane];
+                wsum += w;
+                acc.x += w * v.x;
+                acc.y += w * v.y;
+                acc.z += w * v.z;
+                acc.w += w * v.w;
+            }
+        }
+        const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+        const __nv_bfloat162 lo = __floats2bfloat162_rn(acc.x * inv, acc.y * inv);
+        const __nv_bfloat162 hi = __floats2bfloat162_rn(acc.z * inv, acc.w * inv);
+        uint2 packed;
+        packed.x = *reinterpret_cast<const uint32_t*>(&lo);
+        packed.y = *reinterpret_cast<const uint32_t*>(&hi);
+        reinterpret_cast<uint2*>(m.o + ((static_cast<size_t>(b) * m.s_q + i) * m.h_q + h) * 128)[lane] =
+            packed;
+        if (lane == 0) m.lse[r] = wsum > 0.f ? mx + logf(wsum) : -CUDART_INF_F;
+    }
+}
+
+}  // namespace sdpa10

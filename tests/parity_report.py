@@ -10,7 +10,10 @@ the 2K/4K configs; 512 on the 8K-32K ones), timing the oracle on those rows.
     python tests/parity_report.py [out.jsonl]
 
 prints one markdown table row per (config, mask) and, if a path is given,
-writes the same figures as JSON lines.
+writes the same figures as JSON lines.  A second table times the split-KV
+forward (attn_fwd_split with the library's range count, forward + merge)
+against attn_fwd on few-query, long-key shapes that leave most SMs idle
+unsplit, with parity of the split result on 64 sampled rows per head.
 """
 from __future__ import annotations
 
@@ -30,9 +33,17 @@ import torch  # noqa: E402
 import oracle  # noqa: E402
 from parity import gather_rows, metrics  # noqa: E402
 from scaled_dot_product_10_b200 import attn  # noqa: E402
-from scaled_dot_product_10_b200.workloads import WORKLOADS, sample_rows, workload_qkv  # noqa: E402
+from scaled_dot_product_10_b200.workloads import (  # noqa: E402
+    WORKLOADS, make_qkv, sample_rows, workload_qkv)
 
 SPEC_TFLOPS = 2250.0
+# (name, batch, h_q, h_kv, s_q, s_k, seed): non-causal, N(0,1) BF16 inputs.
+SPLIT_CASES = [
+    ("few_q_b1_h16_q256_k32768", 1, 16, 16, 256, 32768, 1101),
+    ("few_q_b1_h16_q512_k32768", 1, 16, 16, 512, 32768, 1102),
+    ("few_q_b2_h16_q128_k16384", 2, 16, 16, 128, 16384, 1103),
+    ("few_q_gqa_b1_h32_kv4_q256_k65536", 1, 32, 4, 256, 65536, 1104),
+]
 
 
 def measured_peak():
@@ -105,6 +116,38 @@ def main():
                   f"{med:.3f} / {mn:.3f} | {gbs:.0f} | {m['max_abs_o']:.2e} | "
                   f"{m['rel_l2_o']:.2e} | {m['max_abs_lse']:.2e} | "
                   f"{t_oracle:.1f} ({n_rows} rows) |", flush=True)
+    print()
+    print("| split case | n ranges | attn_fwd TFLOPS (ms) | attn_fwd_split TFLOPS (ms) | speed-up | "
+          "alg. GB/s split | max abs dO | rel-L2 O | max abs dLSE |")
+    print("|---|---|---|---|---|---|---|---|---|")
+    for name, b, hq, hkv, sq, sk, seed in SPLIT_CASES:
+        q, k, v = make_qkv(b, hq, hkv, sq, sk, seed=seed)
+        qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+        scale = 1.0 / np.sqrt(128.0)
+        o = torch.empty_like(qd)
+        lse = torch.empty((b, hq, sq), dtype=torch.float32, device="cuda")
+        n = attn.num_splits(b, hq, hkv, sq, sk)
+        ws = torch.empty(attn.split_workspace_bytes(b, hq, sq, n), dtype=torch.uint8, device="cuda")
+        t_plain, _ = time_launches(lambda: attn.attn_fwd(qd, kd, vd, scale=scale, o=o, lse=lse))
+        t_split, _ = time_launches(lambda: attn.attn_fwd_split(qd, kd, vd, scale=scale, n_splits=n,
+                                                               o=o, lse=lse, workspace=ws))
+        rc = attn.attn_status()
+        assert rc == attn.ATTN_OK, attn.attn_strerror(rc)
+        rows = sample_rows(b, hq, sq, 64, seed=seed + 7919)
+        o_ref, l_ref, _ = oracle.attn_fwd(q, k, v, False, scale, rows=rows)
+        oo, ll = gather_rows(o, lse, rows)
+        m = metrics(oo, ll, o_ref, l_ref)
+        flops = 4.0 * b * hq * sq * sk * 128
+        byts = 2 * (b * sq * hq * 128 * 2) + 2 * (b * sk * hkv * 128 * 2) + b * hq * sq * 4
+        tf_p, tf_s = flops / (t_plain * 1e-3) / 1e12, flops / (t_split * 1e-3) / 1e12
+        rec = {"split_case": name, "n_splits": n, "tflops_attn_fwd": tf_p, "ms_attn_fwd": t_plain,
+               "tflops_split": tf_s, "ms_split": t_split, "alg_gbs_split": byts / (t_split * 1e-3) / 1e9,
+               **m}
+        if out:
+            out.write(json.dumps(rec) + "\n")
+        print(f"| {name} | {n} | {tf_p:.1f} ({t_plain:.3f}) | {tf_s:.1f} ({t_split:.3f}) | "
+              f"{t_plain / t_split:.2f}x | {rec['alg_gbs_split']:.0f} | {m['max_abs_o']:.2e} | "
+              f"{m['rel_l2_o']:.2e} | {m['max_abs_lse']:.2e} |", flush=True)
     if out:
         out.close()
 

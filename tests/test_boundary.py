@@ -122,6 +122,58 @@ def test_host_entry_validation(lib):
     assert lib.attn_fwd_host(*args, A + 16, need, None) == attn.ATTN_ERR_ALIGN
 
 
+def test_split_workspace_bytes(lib):
+    b, hq, s, n = 2, 4, 300, 5
+    rows = b * hq * s
+    r = lambda x: (x + 255) // 256 * 256
+    assert lib.attn_fwd_split_workspace_bytes(b, hq, s, n) == r(n * rows * 128 * 4) + n * rows * 4
+    assert lib.attn_fwd_split_workspace_bytes(b, hq, s, 0) == 0
+    assert lib.attn_fwd_split_workspace_bytes(0, hq, s, 2) == 0
+
+
+def test_split_entry_validation(lib):
+    # 256 keys = 2 key blocks: 3 requested ranges become 2.
+    args = (A, A, A, A, A, 1, 2, 2, 256, 256, 128, 0, 0.088)
+    need2 = lib.attn_fwd_split_workspace_bytes(1, 2, 256, 2)
+    assert lib.attn_fwd_split(*args, 0, A, need2, None) == attn.ATTN_ERR_INVALID
+    assert lib.attn_fwd_split(*args, 2, None, need2, None) == attn.ATTN_ERR_INVALID
+    assert lib.attn_fwd_split(*args, 2, A, need2 - 1, None) == attn.ATTN_ERR_INVALID
+    assert lib.attn_fwd_split(*args, 3, A, need2 - 1, None) == attn.ATTN_ERR_INVALID
+    assert lib.attn_fwd_split(*args, 2, A + 16, need2, None) == attn.ATTN_ERR_ALIGN
+    bad = (A, A, A, A, A, 1, 2, 2, 256, 256, 64, 0, 0.088)
+    assert lib.attn_fwd_split(*bad, 2, A, need2, None) == attn.ATTN_ERR_UNSUPPORTED
+    causal_rect = (A, A, A, A, A, 1, 2, 2, 128, 256, 128, 1, 0.088)
+    assert lib.attn_fwd_split(*causal_rect, 2, A, need2, None) == attn.ATTN_ERR_UNSUPPORTED
+
+
+def test_partials_entry_validation(lib):
+    ok = (A, A, A, A, A, 1, 2, 2, 256, 256, 128, 0, 0.088)
+    f = lib.attn_fwd_partials
+    assert f(A, A, A, 0, A, *ok[5:], None) == attn.ATTN_ERR_INVALID
+    assert f(A, A, A, A, 0, *ok[5:], None) == attn.ATTN_ERR_INVALID
+    assert f(A, A, A, A + 8, A, *ok[5:], None) == attn.ATTN_ERR_ALIGN
+    assert f(*ok[:10], 64, 0, 0.088, None) == attn.ATTN_ERR_UNSUPPORTED
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(op=0), attn.ATTN_ERR_INVALID),
+    (dict(lp=0), attn.ATTN_ERR_INVALID),
+    (dict(o=0), attn.ATTN_ERR_INVALID),
+    (dict(lse=0), attn.ATTN_ERR_INVALID),
+    (dict(n=0), attn.ATTN_ERR_INVALID),
+    (dict(s=-1), attn.ATTN_ERR_INVALID),
+    (dict(d=64), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(op=A + 4), attn.ATTN_ERR_ALIGN),
+    (dict(o=A + 8), attn.ATTN_ERR_ALIGN),
+    (dict(lse=A + 2), attn.ATTN_ERR_ALIGN),
+])
+def test_merge_validation_codes(lib, kw, code):
+    a = dict(op=A, lp=A, n=2, b=1, h=2, s=256, d=128, o=A, lse=A)
+    a.update(kw)
+    assert lib.attn_merge_partials(a["op"], a["lp"], a["n"], a["b"], a["h"], a["s"], a["d"],
+                                   a["o"], a["lse"], None) == code
+
+
 def test_python_binding_rejects_wrong_dtype():
     q = torch.zeros(1, 8, 2, 128)
     with pytest.raises(TypeError):
