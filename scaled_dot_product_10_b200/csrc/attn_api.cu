@@ -142,10 +142,17 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     const int rc = init_device(dev, &st);
     if (rc != ATTN_OK) return rc;
 
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!encode_map(&tq, q, h_q, s_q, batch) || !encode_map(&tk, k, h_kv, s_k, batch) ||
         !encode_map(&tv, v, h_kv, s_k, batch))
         return ATTN_ERR_CUDA;
+    // O is stored through a tensor map of the same shape as Q's (unused when
+    // the launch writes FP32 partials instead).
+    if (o != nullptr) {
+        if (!encode_map(&to, o, h_q, s_q, batch)) return ATTN_ERR_CUDA;
+    } else {
+        to = tq;
+    }
 
     FwdParams p{};
     p.batch = batch;
@@ -175,7 +182,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 
     const int grid = p.num_tiles < st->num_sms ? p.num_tiles : st->num_sms;
     attn_fwd_sm100_kernel<<<grid, kThreads, Layout::kAlloc,
-                                       static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, p);
+                                       static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, to, p);
     g_last_launches = 1;
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     return ATTN_OK;

@@ -145,7 +145,8 @@ struct SmemLayout {
                          bSFull = bVEmpty + kVStages,
                          bSFree = bSFull + 2, bPFull = bSFree + 2, bOFull = bPFull + 2,
                          bOEmpty = bOFull + 2, bTurn = bOEmpty + 2, bDrain = bTurn + 1,
-                         kNumBars = bDrain + 2;
+                         bOStaged = bDrain + 2, bOStored = bOStaged + 2,
+                         kNumBars = bOStored + 2;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
@@ -193,9 +194,9 @@ __device__ __forceinline__ void exp_row(const float (&s)[128], uint64_t c2x2, ui
 
 // ------------------------------------------------------------------ softmax
 // One softmax warpgroup: thread r owns query row r of its block (TMEM lane r).
-__device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& wc,
-                                             uint32_t tmem, uint32_t sP, uint32_t bars, int wg,
-                                             int warp_in_wg, int lane) {
+__device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorMap* tm_o,
+                                             const WaitCtx& wc, uint32_t tmem, uint32_t sP,
+                                             uint32_t bars, int wg, int warp_in_wg, int lane) {
     using L = SmemLayout;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
     const int r = warp_in_wg * 32 + lane;
@@ -205,6 +206,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
     const uint32_t b_sfull = bar(L::bSFull + wg), b_sfree = bar(L::bSFree + wg);
     const uint32_t b_pfull = bar(L::bPFull + wg);
     const uint32_t b_ofull = bar(L::bOFull + wg), b_oempty = bar(L::bOEmpty + wg);
+    const uint32_t b_ostaged = bar(L::bOStaged + wg), b_ostored = bar(L::bOStored + wg);
     // This row of P in shared memory (K-major, 128-byte swizzle, two 64-key
     // halves 16 KiB apart): 16-byte chunk c of the row lands at
     // row_base + (c / 8) * 16 KiB + ((c % 8) ^ (r % 8)) * 16.
@@ -220,6 +222,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
     // turn.  Each wait then finds the turn barrier at most one phase short,
     // which its single parity bit can tell apart.
     uint32_t cnt = 0;     // S blocks this warpgroup has processed (all pairs)
+    uint32_t stored = 0;  // O tiles this warpgroup has stored through TMA
     uint32_t rounds = 0;  // alternation rounds before this pair
     PairCursor c;
     c.start(p);
@@ -367,8 +370,10 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
                     if (lane == 0) ptx::mbar_arrive(b_oempty);
                     if (row < p.s_q) p.lse_part[part] = lse_row;
                 } else {
-                    uint4* orow = reinterpret_cast<uint4*>(
-                        p.o + ((static_cast<size_t>(c.b) * p.s_q + row) * p.h_q + c.h) * kHeadDim);
+                    // BF16 O rows go to this block's P buffer (free: the last
+                    // P V has completed) in the tile layout TMA reads, and
+                    // one thread stores the tile with two TMA copies (rows
+                    // past s_q are clipped by the tensor map).
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint32_t ov[32];
@@ -384,21 +389,39 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const WaitCtx& 
                             ptx::f2_unpack(v, lo, hi);
                             w[k] = ptx::pack_bf16x2(lo, hi);
                         }
-                        if (row < p.s_q) {
 #pragma unroll
-                            for (int k = 0; k < 4; ++k)
-                                orow[q * 4 + k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2],
-                                                             w[4 * k + 3]);
+                        for (int k = 0; k < 4; ++k) {
+                            const int cc = 4 * q + k;
+                            ptx::st_shared_v4(
+                                p_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ p_xor) << 4),
+                                w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
                         }
                     }
                     ptx::tc_fence_before();
                     __syncwarp();
                     if (lane == 0) ptx::mbar_arrive(b_oempty);
+                    // Rows staged (all four warps) -> thread 0 stores the tile
+                    // and waits until TMA has read it -> the P buffer is free.
+                    ptx::fence_proxy_async_smem();
+                    __syncwarp();
+                    if (lane == 0) ptx::mbar_arrive(b_ostaged);
+                    if (r == 0) {
+                        if (!wait_bar(b_ostaged, stored & 1, wc)) return;
+                        const uint32_t tile = sP + wg * kTileBytes;
+                        ptx::tma_store_4d(tm_o, tile, 0, c.h, qb * kBlockM, c.b);
+                        ptx::tma_store_4d(tm_o, tile + kHalfTileBytes, 64, c.h, qb * kBlockM, c.b);
+                        ptx::bulk_commit_group();
+                        ptx::bulk_wait_group_read0();
+                        ptx::mbar_arrive(b_ostored);
+                    }
+                    if (!wait_bar_warp(b_ostored, stored & 1, wc)) return;
+                    ++stored;
                     if (row < p.s_q) p.lse[row_id] = lse_row;
                 }
             }
         }
     }
+    if (r == 0) ptx::bulk_wait_group0();  // the last O tile has reached global memory
 }
 
 // ------------------------------------------------------------------ kernel
@@ -406,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
+                          const __grid_constant__ CUtensorMap tm_o,
                           const __grid_constant__ FwdParams p) {
     using L = SmemLayout;
     extern __shared__ uint8_t smem_raw[];
@@ -433,6 +457,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(bar(L::bPFull + i), 4);
             ptx::mbar_init(bar(L::bOFull + i), 1);
             ptx::mbar_init(bar(L::bOEmpty + i), 4);
+            ptx::mbar_init(bar(L::bOStaged + i), 4);  // the 4 warps' rows are staged
+            ptx::mbar_init(bar(L::bOStored + i), 1);  // TMA has read the staged tile
         }
         for (int i = 0; i < kKStages; ++i) {
             ptx::mbar_init(bar(L::bKFull + i), 1);
@@ -452,6 +478,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::prefetch_tmap(&tm_q);
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_v);
+        ptx::prefetch_tmap(&tm_o);
     }
     if (warp == kMmaWarp0) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
@@ -652,7 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp < 8) {
         ptx::reg_alloc<kRegsSoftmax>();
-        softmax_role(p, wc, tmem, sP, bars, warp >> 2, warp & 3, lane);
+        softmax_role(p, &tm_o, wc, tmem, sP, bars, warp >> 2, warp & 3, lane);
     } else {
         ptx::reg_dealloc<kRegsControl>();  // idle warps of the control warpgroup
     }
