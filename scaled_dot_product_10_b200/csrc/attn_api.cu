@@ -172,6 +172,14 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     const size_t per_sec = kL2SectionBytes / (unit_bytes ? unit_bytes : 1);
     const int units_total = batch * h_kv;
     p.units_per_section = static_cast<int>(per_sec < 1 ? 1 : (per_sec > (size_t)units_total ? units_total : per_sec));
+    p.last_section = (units_total - 1) / p.units_per_section;
+    p.last_units = units_total - p.last_section * p.units_per_section;
+    p.div_splits = FastDiv::make(static_cast<uint32_t>(n_splits));
+    p.div_section = FastDiv::make(static_cast<uint32_t>(p.units_per_section) * p.group * p.n_pairs);
+    p.div_rank = FastDiv::make(static_cast<uint32_t>(p.units_per_section) * p.group);
+    p.div_rank_last = FastDiv::make(static_cast<uint32_t>(p.last_units) * p.group);
+    p.div_group = FastDiv::make(static_cast<uint32_t>(p.group));
+    p.div_h_kv = FastDiv::make(static_cast<uint32_t>(h_kv));
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;

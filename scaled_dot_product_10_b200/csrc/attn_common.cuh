@@ -23,6 +23,26 @@ constexpr unsigned kStatusTimeout = 1u;
 // and LSE are unchanged).
 constexpr float kRescaleThresholdLog2 = 8.0f;
 
+// Division by a divisor fixed for the launch, without the hardware's
+// float-reciprocal integer division (whose conversions share the XU pipe
+// with the softmax's ex2): q = (umulhi(n, m) + n) >> s with s = ceil(log2 d)
+// and m = floor(2^32 (2^s - d) / d) + 1 (Granlund and Montgomery, "Division
+// by invariant integers using multiplication", 1994); exact for
+// 0 <= n < 2^31 and 1 <= d < 2^31.
+struct FastDiv {
+    uint32_t d, m, s;
+    __host__ __device__ static FastDiv make(uint32_t d) {
+        uint32_t s = 0;
+        while ((1ull << s) < d) ++s;
+        const uint64_t m = ((1ull << 32) * ((1ull << s) - d)) / d + 1;
+        return FastDiv{d, static_cast<uint32_t>(m), s};
+    }
+    __device__ __forceinline__ int div(int n) const {
+        const uint32_t u = static_cast<uint32_t>(n);
+        return static_cast<int>((__umulhi(u, m) + u) >> s);
+    }
+};
+
 struct FwdParams {
     int batch, h_q, h_kv, s_q, s_k;
     int group;    // h_q / h_kv
@@ -34,6 +54,16 @@ struct FwdParams {
     int units_per_section;  // (batch, kv head) units whose K/V share L2 at once
     int n_splits;           // key ranges per pair (1: the whole key sequence)
     int kb_per_split;       // key blocks per range
+    // Work-item decoding (see PairCursor::decode): sections of
+    // units_per_section (batch, kv head) units, the last one holding
+    // last_units; the divisors the decoding needs.
+    int last_section, last_units;
+    FastDiv div_splits;     // n_splits
+    FastDiv div_section;    // units_per_section * group * n_pairs
+    FastDiv div_rank;       // units_per_section * group
+    FastDiv div_rank_last;  // last_units * group
+    FastDiv div_group;      // group
+    FastDiv div_h_kv;       // h_kv
     float scale_log2;       // scale * log2(e)
     __nv_bfloat16* o;
     float* lse;

@@ -87,22 +87,22 @@ struct PairCursor {
     int n[2];        // key/value blocks each query block of the pair visits (0: none)
 
     __device__ __forceinline__ void decode(const FwdParams& p) {
-        const int u = t / p.n_splits;
+        const int u = p.div_splits.div(t);
         split = t - u * p.n_splits;
         kb0 = split * p.kb_per_split;
         const int kb_end = min(p.n_kb, kb0 + p.kb_per_split);
-        const int per_unit = p.group * p.n_pairs;
-        const int units_total = p.batch * p.h_kv;
         const int G = p.units_per_section;
-        const int sec = u / (G * per_unit);
-        const int r = u - sec * G * per_unit;
-        const int Gs = min(G, units_total - sec * G);
-        const int rank = r / (Gs * p.group);
+        const int sec = p.div_section.div(u);
+        const int r = u - sec * G * p.group * p.n_pairs;
+        const bool last = sec == p.last_section;
+        const int Gs = last ? p.last_units : G;
+        const int rank = last ? p.div_rank_last.div(r) : p.div_rank.div(r);
         const int rem = r - rank * Gs * p.group;
-        const int unit = sec * G + rem / p.group;
-        const int h_local = rem - (rem / p.group) * p.group;
+        const int unit_in_sec = p.div_group.div(rem);
+        const int unit = sec * G + unit_in_sec;
+        const int h_local = rem - unit_in_sec * p.group;
         const int pair = p.n_pairs - 1 - rank;
-        b = unit / p.h_kv;
+        b = p.div_h_kv.div(unit);
         g = unit - b * p.h_kv;
         h = g * p.group + h_local;
         qb0 = 2 * pair;
