@@ -15,9 +15,12 @@
  *   page (section 1, "Query-Key product, softmax normalisation, Value
  *   weighted sum") give them:
  *     1. S[i][j] = scale * sum_c Q[i][c] * K[j][c]          (scores)
- *        causal: S[i][j] = -inf for j > i                  (mask; the
+ *        causal: S[i][j] = -inf for j > i + (s_k - s_q)    (mask; the
  *        intelliparadigm.com AVO page, section 2.2, fuses the mask into
- *        the softmax -- here it is simply applied to S)
+ *        the softmax -- here it is simply applied to S.  The pages only
+ *        use s_q = s_k, where this is j > i; for s_q < s_k the mask is
+ *        aligned to the bottom-right corner, so the last query sees every
+ *        key -- the reading stated in the design notes)
  *     2. m_i = max_j S[i][j];  E = exp(S - m_i);  l_i = sum_j E[i][j];
  *        P = E / l_i        (numerically stable softmax with the scale
  *        applied before the max, as in the AVO page, section 3.1 item 2)
@@ -82,6 +85,7 @@ static void attend_rows(const double *Q, const double *K, const double *V,
     const double *Kb = K + (int64_t)b * s_k * kv_row_stride + (int64_t)g * d;
     const double *Vb = V + (int64_t)b * s_k * kv_row_stride + (int64_t)g * d;
     const int64_t bh = (int64_t)b * h_q + h;
+    const int off = s_k - s_q;  /* causal: row i sees keys 0 .. i + off */
 
     for (int r = r0; r < r1; ++r) {
         const int i = rows ? rows[bh * n_rows + r] : r;
@@ -94,7 +98,7 @@ static void attend_rows(const double *Q, const double *K, const double *V,
                 dot += Qb[(int64_t)i * q_row_stride + c] *
                        Kb[(int64_t)j * kv_row_stride + c];
             Srow[j] = scale * dot;
-            if (causal && j > i) Srow[j] = -INFINITY;
+            if (causal && j > i + off) Srow[j] = -INFINITY;
         }
 
         /* step 2: stable softmax over the row */

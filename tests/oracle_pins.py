@@ -114,6 +114,29 @@ def pin_causal_row0(lib):
             assert abs(lse[bi, hi, 0] - want) < 1e-12, "causal LSE_0 != scale q0.k0"
 
 
+def pin_causal_rectangular_is_square_suffix(lib):
+    """Causal with s_q < s_k (bottom-right alignment): the s_q queries are the
+    last s_q rows of a square causal problem over the same keys, so their O
+    and LSE equal those rows of the square result (pinned above)."""
+    b, h, s_k, s_q, d = 1, 2, 19, 7, 8
+    q_full, k, v = make_qkv(b, h, h, s_k, s_k, seed=41, d=d)
+    q = q_full[:, s_k - s_q:].contiguous()
+    o_sq, l_sq, _ = run(lib, q_full, k, v, True, 0.31)
+    o, l, _ = run(lib, q, k, v, True, 0.31)
+    assert np.max(np.abs(o - o_sq[:, :, s_k - s_q:])) < 1e-12, "rectangular causal != square suffix"
+    assert np.max(np.abs(l - l_sq[:, :, s_k - s_q:])) < 1e-12, "rectangular causal LSE != square suffix"
+
+
+def pin_causal_single_query_sees_every_key(lib):
+    """One query row under the bottom-right causal mask sees all s_k keys:
+    the result equals the non-causal one."""
+    q, k, v = make_qkv(2, 2, 1, 1, 13, seed=42, d=8)
+    o_c, l_c, _ = run(lib, q, k, v, True, 0.5)
+    o_n, l_n, _ = run(lib, q, k, v, False, 0.5)
+    assert np.max(np.abs(o_c - o_n)) < 1e-12 and np.max(np.abs(l_c - l_n)) < 1e-12, \
+        "single causal query does not see every key"
+
+
 def pin_key_shift(lib):
     """Adding one vector c to every key row adds scale*q_i.c to every score of
     row i: O is unchanged and LSE_i moves by scale*q_i.c (both modes)."""
@@ -232,6 +255,7 @@ def pin_row_subset(lib):
 
 ALL_PINS = [
     pin_rows_sum_to_one, pin_identical_v_rows, pin_zero_query, pin_causal_row0,
+    pin_causal_rectangular_is_square_suffix, pin_causal_single_query_sees_every_key,
     pin_key_shift, pin_value_affine, pin_key_permutation, pin_gqa_equals_repeated_mha,
     pin_torch_sdpa_f64, pin_golden_closed_forms, pin_row_subset,
 ]

@@ -40,7 +40,7 @@ def _brute_force(q, k, v, causal, scale):
             for i in range(s_q):
                 scores = []
                 for j in range(s_k):
-                    if causal and j > i:
+                    if causal and j > i + (s_k - s_q):  # bottom-right aligned
                         continue
                     acc = 0.0
                     for c in range(d):
@@ -55,10 +55,11 @@ def _brute_force(q, k, v, causal, scale):
     return o, lse
 
 
-@pytest.mark.parametrize("shape", [(1, 1, 1, 5, 4), (2, 4, 2, 17, 4), (1, 2, 1, 9, 128)])
+@pytest.mark.parametrize("shape", [(1, 1, 1, 5, 5, 4), (2, 4, 2, 17, 17, 4), (1, 2, 1, 9, 9, 128),
+                                   (1, 2, 2, 4, 11, 4), (2, 2, 1, 1, 6, 8)])
 def test_oracle_brute_force(lib, shape):
-    b, h_q, h_kv, s, d = shape
-    q, k, v = make_qkv(b, h_q, h_kv, s, s, seed=31 + s, d=d)
+    b, h_q, h_kv, s_q, s_k, d = shape
+    q, k, v = make_qkv(b, h_q, h_kv, s_q, s_k, seed=31 + s_q + s_k, d=d)
     for causal in (False, True):
         o, lse, _ = oracle.attn_fwd(q, k, v, causal, 0.3, lib=lib)
         ob, lb = _brute_force(q, k, v, causal, 0.3)
@@ -80,8 +81,10 @@ def test_oracle_rejects_bad_arguments(lib):
 # and must fail at least one pin.
 MUTANTS = {
     "dropped_scale": ("Srow[j] = scale * dot;", "Srow[j] = dot;"),
-    "mask_wrong_side": ("if (causal && j > i)", "if (causal && j < i)"),
-    "mask_off_by_one": ("if (causal && j > i)", "if (causal && j > i + 1)"),
+    "mask_wrong_side": ("if (causal && j > i + off)", "if (causal && j < i + off)"),
+    "mask_off_by_one": ("if (causal && j > i + off)", "if (causal && j > i + off + 1)"),
+    "mask_top_left": ("if (causal && j > i + off)", "if (causal && j > i)"),
+    "mask_offset_sign": ("const int off = s_k - s_q;", "const int off = s_q - s_k;"),
     "gqa_modulo_mapping": ("const int g = h / group;", "const int g = h % h_kv;"),
     "transposed_scores": ("dot += Qb[(int64_t)i * q_row_stride + c] *\n                       Kb[(int64_t)j * kv_row_stride + c];",
                           "dot += Qb[(int64_t)j * q_row_stride + c] *\n                       Kb[(int64_t)i * kv_row_stride + c];"),
