@@ -39,7 +39,7 @@ typedef enum {
     ATTN_ERR_INVALID = 1,     /* null pointer, dimension <= 0, h_q % h_kv != 0,
                                  non-finite scale, size beyond the kernel's
                                  32-bit tile indexing, workspace too small */
-    ATTN_ERR_UNSUPPORTED = 2, /* d != 128, or causal with s_q != s_k */
+    ATTN_ERR_UNSUPPORTED = 2, /* d != 128, or causal with s_q > s_k */
     ATTN_ERR_ALIGN = 3,       /* a q/k/v/o pointer not 16-byte aligned (TMA),
                                  or lse not 4-byte aligned */
     ATTN_ERR_CUDA = 4,        /* a CUDA runtime/driver call failed (no device,
@@ -60,8 +60,10 @@ typedef enum {
  *   o    device, bf16 [batch, s_q, h_q,  d] contiguous (written)
  *   lse  device, fp32 [batch, h_q, s_q]     contiguous (written)
  *   d     must be 128
- *   causal  0: full attention; 1: key j is visible to query i iff j <= i
- *           (requires s_q == s_k)
+ *   causal  0: full attention; 1: key j is visible to query i iff
+ *           j <= i + (s_k - s_q) -- the mask aligned to the bottom-right
+ *           corner, so the last query sees every key (j <= i when
+ *           s_q == s_k); requires s_q <= s_k
  *   scale   multiplies Q K^T before the softmax (usually 1/sqrt(d))
  *
  * The caller owns every buffer; the call allocates nothing.  o and lse must

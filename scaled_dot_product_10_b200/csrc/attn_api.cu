@@ -107,7 +107,7 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
     if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
     if (!(scale > 0.f)) return ATTN_ERR_UNSUPPORTED;
     if (causal != 0 && causal != 1) return ATTN_ERR_INVALID;
-    if (causal && s_q != s_k) return ATTN_ERR_UNSUPPORTED;
+    if (causal && s_q > s_k) return ATTN_ERR_UNSUPPORTED;  // a row would see no key
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
         !aligned(lse, 4))
         return ATTN_ERR_ALIGN;
@@ -164,6 +164,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.n_qb = (s_q + kBlockM - 1) / kBlockM;
     p.n_kb = (s_k + kBlockN - 1) / kBlockN;
     p.causal = causal;
+    p.causal_offset = s_k - s_q;
     p.n_pairs = (p.n_qb + 1) / 2;
     p.n_splits = n_splits;
     p.kb_per_split = kb_per_split;
@@ -214,6 +215,7 @@ int launch_merge(const float* o_part, const float* lse_part, int n_parts, int ba
     m.keys_per_part = keys_per_part;
     m.s_k = s_k;
     m.causal = causal;
+    m.causal_offset = s_k - s_q;
     m.o = static_cast<__nv_bfloat16*>(o);
     m.lse = lse;
     const size_t rows = static_cast<size_t>(batch) * h_q * s_q;

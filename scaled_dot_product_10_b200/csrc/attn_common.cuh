@@ -50,6 +50,7 @@ struct FwdParams {
     int n_kb;     // ceil(s_k / 128)
     int n_pairs;  // ceil(n_qb / 2): CTA tiles per (batch, head)
     int causal;
+    int causal_offset;      // s_k - s_q: causal row i sees keys 0 .. i + causal_offset
     int num_tiles;          // work items: pairs x n_splits
     int units_per_section;  // (batch, kv head) units whose K/V share L2 at once
     int n_splits;           // key ranges per pair (1: the whole key sequence)

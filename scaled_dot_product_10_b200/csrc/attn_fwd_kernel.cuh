@@ -106,9 +106,12 @@ struct PairCursor {
         g = unit - b * p.h_kv;
         h = g * p.group + h_local;
         qb0 = 2 * pair;
-        // Causal (s_q == s_k): rows of block qb see key blocks 0..qb.
-        const int vis0 = p.causal ? min(kb_end, qb0 + 1) : kb_end;
-        const int vis1 = (qb0 + 1 < p.n_qb) ? (p.causal ? min(kb_end, qb0 + 2) : kb_end) : 0;
+        // Causal (bottom-right aligned, s_q <= s_k): the last row of block
+        // qb, min(128 qb + 127, s_q - 1), sees keys up to row + s_k - s_q.
+        const int last0 = (min(qb0 * kBlockM + kBlockM - 1, p.s_q - 1) + p.causal_offset) / kBlockN;
+        const int last1 = (min(qb0 * kBlockM + 2 * kBlockM - 1, p.s_q - 1) + p.causal_offset) / kBlockN;
+        const int vis0 = p.causal ? min(kb_end, last0 + 1) : kb_end;
+        const int vis1 = (qb0 + 1 < p.n_qb) ? (p.causal ? min(kb_end, last1 + 1) : kb_end) : 0;
         n[0] = max(0, vis0 - kb0);
         n[1] = max(0, vis1 - kb0);
     }
@@ -254,11 +257,12 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
             if (lane == 0) ptx::mbar_arrive(b_sfree);
 
             const int kv0 = (c.kb0 + j) * kBlockN;
-            const bool diag = p.causal && (kv0 + kBlockN - 1 > qb * kBlockM);
+            const bool diag = p.causal && (kv0 + kBlockN - 1 > qb * kBlockM + p.causal_offset);
             const bool masked = diag || kv0 + kBlockN > p.s_k;
             if (masked) {
                 const int lim_tail = p.s_k - kv0;                           // keys >= s_k
-                const int lim_causal = p.causal ? row - kv0 + 1 : kBlockN;  // keys > row
+                // keys past row + s_k - s_q
+                const int lim_causal = p.causal ? row + p.causal_offset - kv0 + 1 : kBlockN;
                 const int lim = min(lim_tail, lim_causal);
 #pragma unroll
                 for (int k = 0; k < 128; ++k)

@@ -24,10 +24,11 @@ struct MergeParams {
     int batch, h_q, s_q;
     // Key ranges of keys_per_part keys each, over s_k keys: range r holds
     // keys [r * keys_per_part, (r + 1) * keys_per_part).  A range that holds
-    // no key of the row (past s_k, or past the row under the causal mask) is
-    // not read.  keys_per_part = 0: every part is read for every row (a part
+    // no key of the row (past s_k, or past row + causal_offset under the
+    // causal mask) is not read.  keys_per_part = 0: every part is read for every row (a part
     // with LSE = -inf then carries no weight).
     int keys_per_part, s_k, causal;
+    int causal_offset;  // s_k - s_q: causal row i sees keys 0 .. i + causal_offset
     __nv_bfloat16* o;  // [batch][s_q][h_q][128]
     float* lse;        // [batch][h_q][s_q]
 };
@@ -47,7 +48,7 @@ __global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const MergePa
         int nv = m.n_parts;
         if (m.keys_per_part > 0) {
             nv = min(nv, (m.s_k + m.keys_per_part - 1) / m.keys_per_part);
-            if (m.causal) nv = min(nv, i / m.keys_per_part + 1);
+            if (m.causal) nv = min(nv, (i + m.causal_offset) / m.keys_per_part + 1);
         }
         float mx = -CUDART_INF_F;
         for (int s = 0; s < nv; ++s) mx = fmaxf(mx, m.lse_part[static_cast<size_t>(s) * rows + r]);

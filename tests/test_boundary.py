@@ -73,7 +73,7 @@ def call(lib, q=A, k=A, v=A, o=None, lse=None, b=1, hq=2, hkv=2, sq=256, sk=256,
     (dict(hq=6, hkv=4), attn.ATTN_ERR_INVALID),
     (dict(d=64), attn.ATTN_ERR_UNSUPPORTED),
     (dict(d=256), attn.ATTN_ERR_UNSUPPORTED),
-    (dict(causal=1, sq=256, sk=512), attn.ATTN_ERR_UNSUPPORTED),
+    (dict(causal=1, sq=512, sk=256), attn.ATTN_ERR_UNSUPPORTED),
     (dict(causal=2), attn.ATTN_ERR_INVALID),
     (dict(scale=float("nan")), attn.ATTN_ERR_INVALID),
     (dict(scale=float("inf")), attn.ATTN_ERR_INVALID),
@@ -142,7 +142,7 @@ def test_split_entry_validation(lib):
     assert lib.attn_fwd_split(*args, 2, A + 16, need2, None) == attn.ATTN_ERR_ALIGN
     bad = (A, A, A, A, A, 1, 2, 2, 256, 256, 64, 0, 0.088)
     assert lib.attn_fwd_split(*bad, 2, A, need2, None) == attn.ATTN_ERR_UNSUPPORTED
-    causal_rect = (A, A, A, A, A, 1, 2, 2, 128, 256, 128, 1, 0.088)
+    causal_rect = (A, A, A, A, A, 1, 2, 2, 256, 128, 128, 1, 0.088)
     assert lib.attn_fwd_split(*causal_rect, 2, A, need2, None) == attn.ATTN_ERR_UNSUPPORTED
 
 

@@ -47,6 +47,20 @@ def test_noncausal_rectangular(s_q, s_k):
     check(q, k, v, False, SCALE, what=f"s_q={s_q} s_k={s_k}")
 
 
+@pytest.mark.parametrize("b,hq,hkv,s_q,s_k", [
+    (1, 4, 4, 100, 1000),    # bottom-right diagonal inside a key block
+    (1, 2, 2, 129, 1000),    # ragged queries, two query blocks
+    (2, 8, 2, 384, 4096),    # GQA, three query blocks (an odd pair)
+    (1, 16, 16, 1, 4096),    # one query row (decode) sees every key
+    (1, 4, 1, 640, 643),     # offset 3: diagonal blocks straddle key blocks
+])
+def test_causal_rectangular(b, hq, hkv, s_q, s_k):
+    # Causal with fewer queries than keys: query i sees keys 0 .. i + s_k - s_q.
+    q, k, v = make_qkv(b, hq, hkv, s_q, s_k, seed=6800 + s_q + s_k)
+    rows = None if b * hq * s_q <= 8192 else sample_rows(b, hq, s_q, 64, seed=6801)
+    check(q, k, v, True, SCALE, rows=rows, what=f"causal {s_q}x{s_k}")
+
+
 @pytest.mark.parametrize("h_q,h_kv", [(16, 2), (16, 1), (8, 8), (6, 3), (4, 1)])
 @pytest.mark.parametrize("causal", [False, True])
 def test_head_sharing_small(h_q, h_kv, causal):

@@ -49,6 +49,10 @@ def run_split(q, k, v, causal, n_splits):
     (2, 4, 4, 64, 4096, False, 32),      # one key block per range
     (1, 2, 2, 1, 300, False, 3),         # a single query row
     (3, 6, 3, 200, 2000, False, 2),
+    (1, 16, 16, 64, 32768, True, None),  # causal decode-like: bottom-right mask
+    (2, 8, 2, 1, 8192, True, 5),         # one query row, causal
+    (1, 4, 4, 300, 5000, True, 3),       # causal, ranges that early rows cannot see
+    (1, 4, 4, 200, 300, True, 3),        # offset 100 inside the first key block
 ])
 def test_split_matches_oracle(b, hq, hkv, sq, sk, causal, n):
     q, k, v = make_qkv(b, hq, hkv, sq, sk, seed=7100 + sq + sk)
