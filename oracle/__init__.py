@@ -47,7 +47,7 @@ def load(path: str | None = None):
     lib.oracle_attn_fwd_f64.argtypes = [
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
-        ctypes.c_int, ctypes.c_double,
+        ctypes.c_int, ctypes.c_int, ctypes.c_double,
         ctypes.c_void_p, ctypes.c_int,
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
     ]
@@ -73,13 +73,16 @@ def _as_bits(x) -> np.ndarray:
     return np.ascontiguousarray(x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16))
 
 
-def attn_fwd(q, k, v, causal: bool, scale: float, rows=None, want_p: bool = False, lib=None):
+def attn_fwd(q, k, v, causal: bool, scale: float, rows=None, want_p: bool = False, lib=None,
+             window_left: int = -1):
     """Run the oracle.
 
     q: [batch, s_q, h_q, d] bf16 (torch tensor or uint16 bits);
     k, v: [batch, s_k, h_kv, d].
     rows: None (every query row) or an int array [batch, h_q, n_rows] of the
     query indices to evaluate per (batch, head).
+    window_left: -1 (none) or, with causal, the sliding window: row i sees
+    keys i + s_k - s_q - window_left .. i + s_k - s_q.
 
     Returns (o, lse, p): o [batch, h_q, n_rows, d] float64,
     lse [batch, h_q, n_rows] float64 (natural log), p [batch, h_q, n_rows, s_k]
@@ -104,7 +107,7 @@ def attn_fwd(q, k, v, causal: bool, scale: float, rows=None, want_p: bool = Fals
     lib = lib or load()
     rc = lib.oracle_attn_fwd_f64(
         qb.ctypes.data, kb.ctypes.data, vb.ctypes.data,
-        batch, h_q, h_kv, s_q, s_k, d, int(bool(causal)), float(scale),
+        batch, h_q, h_kv, s_q, s_k, d, int(bool(causal)), int(window_left), float(scale),
         None if rows_arr is None else rows_arr.ctypes.data, n_rows,
         o.ctypes.data, lse.ctypes.data, None if p is None else p.ctypes.data)
     if rc != 0:

@@ -21,6 +21,10 @@
  *        use s_q = s_k, where this is j > i; for s_q < s_k the mask is
  *        aligned to the bottom-right corner, so the last query sees every
  *        key -- the reading stated in the design notes)
+ *        sliding window (window_left >= 0, causal only): also
+ *        S[i][j] = -inf for j < i + (s_k - s_q) - window_left, so row i
+ *        sees the window_left + 1 keys ending at its diagonal (the local
+ *        window variant; the reading is stated in the design notes)
  *     2. m_i = max_j S[i][j];  E = exp(S - m_i);  l_i = sum_j E[i][j];
  *        P = E / l_i        (numerically stable softmax with the scale
  *        applied before the max, as in the AVO page, section 3.1 item 2)
@@ -73,7 +77,7 @@ static double *decode_bf16(const uint16_t *src, int64_t n)
  * S is materialised for the chunk: n_chunk x s_k doubles. */
 static void attend_rows(const double *Q, const double *K, const double *V,
                         int b, int h, int h_q, int h_kv, int s_q, int s_k,
-                        int d, int causal, double scale,
+                        int d, int causal, int window_left, double scale,
                         const int32_t *rows, int r0, int r1, int n_rows,
                         double *o, double *lse, double *p, double *S)
 {
@@ -99,6 +103,7 @@ static void attend_rows(const double *Q, const double *K, const double *V,
                        Kb[(int64_t)j * kv_row_stride + c];
             Srow[j] = scale * dot;
             if (causal && j > i + off) Srow[j] = -INFINITY;
+            if (window_left >= 0 && j < i + off - window_left) Srow[j] = -INFINITY;
         }
 
         /* step 2: stable softmax over the row */
@@ -130,7 +135,7 @@ static void attend_rows(const double *Q, const double *K, const double *V,
 
 int oracle_attn_fwd_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                         int batch, int h_q, int h_kv, int s_q, int s_k, int d,
-                        int causal, double scale,
+                        int causal, int window_left, double scale,
                         const int32_t *rows, int n_rows,
                         double *o, double *lse, double *p)
 {
@@ -144,6 +149,8 @@ int oracle_attn_fwd_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     }
     /* A causal row must see at least one key (row i sees keys 0..i). */
     if (causal && s_q > s_k) return -6;
+    /* A window is a causal mask's lower edge. */
+    if (window_left < -1 || (window_left >= 0 && !causal)) return -8;
 
     double *Q = decode_bf16(q, (int64_t)batch * s_q * h_q * d);
     double *K = decode_bf16(k, (int64_t)batch * s_k * h_kv * d);
@@ -170,7 +177,7 @@ int oracle_attn_fwd_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
             const int b = (int)(bh / h_q), h = (int)(bh % h_q);
             const int r0 = cidx * chunk;
             const int r1 = r0 + chunk < n_rows ? r0 + chunk : n_rows;
-            attend_rows(Q, K, V, b, h, h_q, h_kv, s_q, s_k, d, causal, scale,
+            attend_rows(Q, K, V, b, h, h_q, h_kv, s_q, s_k, d, causal, window_left, scale,
                         rows, r0, r1, n_rows, o, lse, p, S);
         }
         free(S);

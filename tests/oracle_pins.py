@@ -50,6 +50,11 @@ def run(lib, q, k, v, causal, scale, rows=None, want_p=False):
     return oracle.attn_fwd(q, k, v, causal, scale, rows=rows, want_p=want_p, lib=lib)
 
 
+def run_w(lib, q, k, v, scale, window_left):
+    """Causal with a sliding window of window_left keys before the diagonal."""
+    return oracle.attn_fwd(q, k, v, True, scale, lib=lib, window_left=window_left)
+
+
 # ---------------------------------------------------------------------------
 
 
@@ -135,6 +140,48 @@ def pin_causal_single_query_sees_every_key(lib):
     o_n, l_n, _ = run(lib, q, k, v, False, 0.5)
     assert np.max(np.abs(o_c - o_n)) < 1e-12 and np.max(np.abs(l_c - l_n)) < 1e-12, \
         "single causal query does not see every key"
+
+
+def pin_window_covering_every_key_is_causal(lib):
+    """A sliding window at least as wide as the key sequence removes nothing
+    the causal mask keeps."""
+    q, k, v = make_qkv(1, 2, 2, 9, 17, seed=43, d=8)
+    o_w, l_w, _ = run_w(lib, q, k, v, 0.37, 17)
+    o_c, l_c, _ = run(lib, q, k, v, True, 0.37)
+    assert np.max(np.abs(o_w - o_c)) < 1e-12 and np.max(np.abs(l_w - l_c)) < 1e-12, \
+        "full-width window differs from causal"
+
+
+def pin_window_zero_keeps_the_diagonal_key(lib):
+    """window_left = 0: row i sees only key i + s_k - s_q, so O_i is that V row
+    and LSE_i = scale * q_i . k_(i + s_k - s_q)."""
+    b, h, s_q, s_k, d = 1, 2, 6, 10, 8
+    q, k, v = make_qkv(b, h, h, s_q, s_k, seed=44, d=d)
+    scale = 0.29
+    o, lse, _ = run_w(lib, q, k, v, scale, 0)
+    qq, kk, vv = f64(q), f64(k), f64(v)
+    for hi in range(h):
+        for i in range(s_q):
+            j = i + s_k - s_q
+            assert np.max(np.abs(o[0, hi, i] - vv[0, j, hi])) < 1e-12, "window 0: O != V_diag"
+            want = scale * float(np.dot(qq[0, i, hi], kk[0, j, hi]))
+            assert abs(lse[0, hi, i] - want) < 1e-12, "window 0: LSE != scale q.k_diag"
+
+
+def pin_window_row_is_attention_over_its_keys(lib):
+    """Row i under a window of W sees exactly the keys lo..hi with
+    hi = i + s_k - s_q and lo = max(0, hi - W): its O and LSE equal plain
+    (non-causal) attention of that row over K[lo:hi+1], V[lo:hi+1]."""
+    b, h, s_q, s_k, d, W = 1, 2, 12, 15, 8, 4
+    q, k, v = make_qkv(b, h, 1, s_q, s_k, seed=45, d=d)
+    o, lse, _ = run_w(lib, q, k, v, 0.41, W)
+    for i in (0, 1, 5, 11):
+        hi = i + s_k - s_q
+        lo = max(0, hi - W)
+        o1, l1, _ = run(lib, q[:, i:i + 1].contiguous(), k[:, lo:hi + 1].contiguous(),
+                        v[:, lo:hi + 1].contiguous(), False, 0.41)
+        assert np.max(np.abs(o[:, :, i] - o1[:, :, 0])) < 1e-12, "window row != attention over its keys"
+        assert np.max(np.abs(lse[:, :, i] - l1[:, :, 0])) < 1e-12, "window LSE != attention over its keys"
 
 
 def pin_key_shift(lib):
@@ -256,6 +303,8 @@ def pin_row_subset(lib):
 ALL_PINS = [
     pin_rows_sum_to_one, pin_identical_v_rows, pin_zero_query, pin_causal_row0,
     pin_causal_rectangular_is_square_suffix, pin_causal_single_query_sees_every_key,
+    pin_window_covering_every_key_is_causal, pin_window_zero_keeps_the_diagonal_key,
+    pin_window_row_is_attention_over_its_keys,
     pin_key_shift, pin_value_affine, pin_key_permutation, pin_gqa_equals_repeated_mha,
     pin_torch_sdpa_f64, pin_golden_closed_forms, pin_row_subset,
 ]

@@ -24,7 +24,7 @@ def test_oracle_pin(lib, pin):
     pin(lib)
 
 
-def _brute_force(q, k, v, causal, scale):
+def _brute_force(q, k, v, causal, scale, window_left=-1):
     """Per-element scalar evaluation in pure Python floats (tiny shapes only)."""
     qq = q.float().double().tolist()
     kk = k.float().double().tolist()
@@ -41,6 +41,8 @@ def _brute_force(q, k, v, causal, scale):
                 scores = []
                 for j in range(s_k):
                     if causal and j > i + (s_k - s_q):  # bottom-right aligned
+                        continue
+                    if window_left >= 0 and j < i + (s_k - s_q) - window_left:
                         continue
                     acc = 0.0
                     for c in range(d):
@@ -65,6 +67,17 @@ def test_oracle_brute_force(lib, shape):
         ob, lb = _brute_force(q, k, v, causal, 0.3)
         assert np.max(np.abs(o - ob)) < 1e-12
         assert np.max(np.abs(lse - lb)) < 1e-12
+
+
+@pytest.mark.parametrize("shape,window", [((1, 2, 1, 7, 7, 4), 2), ((2, 2, 2, 5, 12, 8), 3),
+                                          ((1, 1, 1, 9, 9, 4), 0)])
+def test_oracle_brute_force_window(lib, shape, window):
+    b, h_q, h_kv, s_q, s_k, d = shape
+    q, k, v = make_qkv(b, h_q, h_kv, s_q, s_k, seed=51 + s_q + window, d=d)
+    o, lse, _ = oracle.attn_fwd(q, k, v, True, 0.3, lib=lib, window_left=window)
+    ob, lb = _brute_force(q, k, v, True, 0.3, window_left=window)
+    assert np.max(np.abs(o - ob)) < 1e-12
+    assert np.max(np.abs(lse - lb)) < 1e-12
 
 
 def test_oracle_rejects_bad_arguments(lib):
@@ -97,6 +110,8 @@ MUTANTS = {
     "lse_log2": ("m + log(l);", "m + log2(l);"),
     "k_used_as_v": ("const double *vrow = Vb +", "const double *vrow = Kb +"),
     "mask_to_zero": ("Srow[j] = -INFINITY;", "Srow[j] = 0.0;"),
+    "window_off_by_one": ("j < i + off - window_left)", "j < i + off - window_left + 1)"),
+    "window_wrong_side": ("j < i + off - window_left)", "j > i + off - window_left)"),
     "bf16_decode_shift": ("((uint32_t)bits) << 16", "((uint32_t)bits) << 15"),
 }
 
