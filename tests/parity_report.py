@@ -7,7 +7,7 @@ minimum), and compares O and LSE with the FP64 oracle on the same rows the
 parity tests use (all rows of the tiny config; 256 sampled rows per head on
 the 2K/4K configs; 512 on the 8K-32K ones), timing the oracle on those rows.
 
-    python tests/parity_report.py [out.jsonl]
+    python tests/parity_report.py [--split-only] [out.jsonl]
 
 prints one markdown table row per (config, mask) and, if a path is given,
 writes the same figures as JSON lines.  A second table times the split-KV
@@ -75,14 +75,17 @@ def time_launches(f, warmup=3, n=20):
 
 
 def main():
-    out = open(sys.argv[1], "w") if len(sys.argv) > 1 else None
+    argv = [a for a in sys.argv[1:] if a != "--split-only"]
+    split_only = len(argv) != len(sys.argv) - 1
+    out = open(argv[0], "w") if argv else None
     peak, peak_src = measured_peak()
     threads = oracle.num_threads()
-    print(f"| config | mode | TFLOPS (median) | % of 2250 | % of {peak_src} {peak} | "
-          "ms median / min | alg. GB/s | max abs dO | rel-L2 O | max abs dLSE | "
-          f"oracle s (rows) / {threads} threads |")
-    print("|---|---|---|---|---|---|---|---|---|---|---|")
-    for name, w in WORKLOADS.items():
+    if not split_only:
+        print(f"| config | mode | TFLOPS (median) | % of 2250 | % of {peak_src} {peak} | "
+              "ms median / min | alg. GB/s | max abs dO | rel-L2 O | max abs dLSE | "
+              f"oracle s (rows) / {threads} threads |")
+        print("|---|---|---|---|---|---|---|---|---|---|---|")
+    for name, w in ([] if split_only else WORKLOADS.items()):
         q, k, v = workload_qkv(w)
         qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
         o = torch.empty_like(qd)
@@ -116,7 +119,8 @@ def main():
                   f"{med:.3f} / {mn:.3f} | {gbs:.0f} | {m['max_abs_o']:.2e} | "
                   f"{m['rel_l2_o']:.2e} | {m['max_abs_lse']:.2e} | "
                   f"{t_oracle:.1f} ({n_rows} rows) |", flush=True)
-    print()
+    if not split_only:
+        print()
     print("| split case | n ranges | attn_fwd TFLOPS (ms) | attn_fwd_split TFLOPS (ms) | speed-up | "
           "alg. GB/s split | max abs dO | rel-L2 O | max abs dLSE |")
     print("|---|---|---|---|---|---|---|---|---|")
