@@ -184,6 +184,21 @@ def pin_window_row_is_attention_over_its_keys(lib):
         assert np.max(np.abs(lse[:, :, i] - l1[:, :, 0])) < 1e-12, "window LSE != attention over its keys"
 
 
+def pin_key_split_merge(lib):
+    """Softmax over a key set cut into two ranges: with (O_r, LSE_r) the
+    results over each range, LSE = log(exp LSE_1 + exp LSE_2) and
+    O = sum_r exp(LSE_r - LSE) O_r reproduce the whole set's O and LSE."""
+    q, k, v = make_qkv(2, 3, 1, 5, 14, seed=46, d=8)
+    o, lse, _ = run(lib, q, k, v, False, 0.33)
+    o1, l1, _ = run(lib, q, k[:, :6].contiguous(), v[:, :6].contiguous(), False, 0.33)
+    o2, l2, _ = run(lib, q, k[:, 6:].contiguous(), v[:, 6:].contiguous(), False, 0.33)
+    m = np.maximum(l1, l2)
+    lse_m = m + np.log(np.exp(l1 - m) + np.exp(l2 - m))
+    o_m = np.exp(l1 - lse_m)[..., None] * o1 + np.exp(l2 - lse_m)[..., None] * o2
+    assert np.max(np.abs(lse_m - lse)) < 1e-12, "key-range LSEs do not combine to the LSE"
+    assert np.max(np.abs(o_m - o)) < 1e-12, "key-range outputs do not combine to O"
+
+
 def pin_key_shift(lib):
     """Adding one vector c to every key row adds scale*q_i.c to every score of
     row i: O is unchanged and LSE_i moves by scale*q_i.c (both modes)."""
@@ -304,7 +319,7 @@ ALL_PINS = [
     pin_rows_sum_to_one, pin_identical_v_rows, pin_zero_query, pin_causal_row0,
     pin_causal_rectangular_is_square_suffix, pin_causal_single_query_sees_every_key,
     pin_window_covering_every_key_is_causal, pin_window_zero_keeps_the_diagonal_key,
-    pin_window_row_is_attention_over_its_keys,
+    pin_window_row_is_attention_over_its_keys, pin_key_split_merge,
     pin_key_shift, pin_value_affine, pin_key_permutation, pin_gqa_equals_repeated_mha,
     pin_torch_sdpa_f64, pin_golden_closed_forms, pin_row_subset,
 ]

@@ -140,6 +140,11 @@ def test_split_entry_validation(lib):
     assert lib.attn_fwd_split(*args, 2, A, need2 - 1, None) == attn.ATTN_ERR_INVALID
     assert lib.attn_fwd_split(*args, 3, A, need2 - 1, None) == attn.ATTN_ERR_INVALID
     assert lib.attn_fwd_split(*args, 2, A + 16, need2, None) == attn.ATTN_ERR_ALIGN
+    # A workspace of exactly the documented size passes validation (the call
+    # then fails only for want of a device, or runs if there is one).
+    if not torch.cuda.is_available():
+        assert lib.attn_fwd_split(*args, 2, A, need2, None) == attn.ATTN_ERR_CUDA
+        assert lib.attn_fwd_split(*args, 3, A, need2, None) == attn.ATTN_ERR_CUDA
     bad = (A, A, A, A, A, 1, 2, 2, 256, 256, 64, 0, 0.088)
     assert lib.attn_fwd_split(*bad, 2, A, need2, None) == attn.ATTN_ERR_UNSUPPORTED
     causal_rect = (A, A, A, A, A, 1, 2, 2, 256, 128, 128, 1, 0.088)
