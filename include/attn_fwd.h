@@ -6,8 +6,10 @@
  * section 1; the three steps of the bjdmk.com.cn survey page, section 1):
  *
  *     S   = scale * Q K^T                  (per batch and query head)
- *     S   = S with S[i][j] = -inf for j > i          (causal mode only; the
- *           mask of the intelliparadigm.com AVO page, section 2.2)
+ *     S   = S with S[i][j] = -inf for j > i + (s_k - s_q)
+ *           (causal mode only, s_q <= s_k: the mask of the
+ *           intelliparadigm.com AVO page, section 2.2, aligned to the
+ *           bottom-right corner; j > i when s_q == s_k)
  *     O   = softmax_rows(S) V
  *     LSE = log(sum_j exp(S[i][j]))        (natural log, per query row)
  *
@@ -37,8 +39,9 @@ extern "C" {
 typedef enum {
     ATTN_OK = 0,
     ATTN_ERR_INVALID = 1,     /* null pointer, dimension <= 0, h_q % h_kv != 0,
-                                 non-finite scale, size beyond the kernel's
-                                 32-bit tile indexing, workspace too small */
+                                 non-finite scale, causal not 0 or 1, size
+                                 beyond the kernel's 32-bit tile indexing,
+                                 workspace too small */
     ATTN_ERR_UNSUPPORTED = 2, /* d != 128, or causal with s_q > s_k */
     ATTN_ERR_ALIGN = 3,       /* a q/k/v/o pointer not 16-byte aligned (TMA),
                                  or lse not 4-byte aligned */
@@ -64,7 +67,9 @@ typedef enum {
  *           j <= i + (s_k - s_q) -- the mask aligned to the bottom-right
  *           corner, so the last query sees every key (j <= i when
  *           s_q == s_k); requires s_q <= s_k
- *   scale   multiplies Q K^T before the softmax (usually 1/sqrt(d))
+ *   scale   multiplies Q K^T before the softmax (usually 1/sqrt(d)); any
+ *           finite value, including 0 (uniform weights over the visible
+ *           keys) and negative values
  *
  * The caller owns every buffer; the call allocates nothing.  o and lse must
  * not overlap the inputs.  q/k/v/o must be 16-byte aligned, lse 4-byte

@@ -105,7 +105,6 @@ int validate(const void* q, const void* k, const void* v, const void* o, const f
     int rc = validate_sizes(batch, h_q, h_kv, s_q, s_k, d);
     if (rc != ATTN_OK) return rc;
     if (!std::isfinite(scale)) return ATTN_ERR_INVALID;
-    if (!(scale > 0.f)) return ATTN_ERR_UNSUPPORTED;
     if (causal != 0 && causal != 1) return ATTN_ERR_INVALID;
     if (causal && s_q > s_k) return ATTN_ERR_UNSUPPORTED;  // a row would see no key
     if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
@@ -181,7 +180,11 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.div_rank_last = FastDiv::make(static_cast<uint32_t>(p.last_units) * p.group);
     p.div_group = FastDiv::make(static_cast<uint32_t>(p.group));
     p.div_h_kv = FastDiv::make(static_cast<uint32_t>(h_kv));
-    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    // The kernel exponentiates 2^((s - m) c) with c > 0: a negative scale
+    // negates the scores on the tensor core instead (see FwdParams).
+    const double c = std::fabs(static_cast<double>(scale)) * 1.4426950408889634;
+    p.scale_log2 = static_cast<float>(c < 1e-30 ? 1e-30 : c);
+    p.idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, 0, 0) | (scale < 0.f ? kIdescNegateA : 0u);
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
     p.o_part = o_part;
@@ -377,7 +380,7 @@ extern "C" const char* attn_strerror(int code) {
     switch (code) {
         case ATTN_OK: return "success";
         case ATTN_ERR_INVALID: return "invalid argument";
-        case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (d must be 128; causal needs s_q == s_k; scale must be > 0)";
+        case ATTN_ERR_UNSUPPORTED: return "unsupported configuration (d must be 128; causal needs s_q <= s_k)";
         case ATTN_ERR_ALIGN: return "misaligned pointer (q/k/v/o need 16 bytes, lse 4 bytes)";
         case ATTN_ERR_CUDA: return "CUDA runtime or driver error";
         case ATTN_ERR_TIMEOUT: return "a kernel gave up a bounded device-side wait";

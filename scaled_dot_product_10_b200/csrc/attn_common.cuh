@@ -65,7 +65,15 @@ struct FwdParams {
     FastDiv div_rank_last;  // last_units * group
     FastDiv div_group;      // group
     FastDiv div_h_kv;       // h_kv
-    float scale_log2;       // scale * log2(e)
+    // |scale| * log2(e) (at least 1e-30, see below).  A negative scale is
+    // carried by the sign of the scores themselves: the Q K^T instruction
+    // descriptor negates A, so the tensor core produces -Q K^T and the
+    // softmax always works with a positive factor.  Scale 0 runs with the
+    // factor 1e-30: every exponent is then below 2^-90 and every weight
+    // rounds to exactly 1 in FP32, the uniform softmax, while masked
+    // scores (-inf) still give weight 0 (0 * -inf would be NaN).
+    float scale_log2;
+    uint32_t idesc_qk;      // instruction descriptor of S = (+/-) Q K^T
     __nv_bfloat16* o;
     float* lse;
     // Split-KV partials (null unless n_splits > 1 or a split launch): per key

@@ -573,7 +573,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         ptx::reg_dealloc<kRegsControl>();
         if (lane == 0) {
             const int i = (warp == kMmaWarp0) ? 0 : 1;  // query block this lane serves
-            constexpr uint32_t kIdescQK = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);
+            const uint32_t idesc_qk = p.idesc_qk;
             constexpr uint32_t kIdescPV = idesc_bf16_f32(kBlockM, kHeadDim, 0, 1);
             uint32_t k_used = 0, v_used = 0;  // K / V tiles passed (used or skipped)
             uint32_t started = 0;             // pairs in which query block i was active
@@ -616,7 +616,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // K-major, 128-byte swizzle: 16 BF16 (32 bytes) per step
                     // inside a 64-column half; the second half is 16 KiB on.
                     const uint32_t off = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
-                    ptx::mma_ss(s_tm, desc_from_lo(q_lo + off), desc_from_lo(ka + off), kIdescQK,
+                    ptx::mma_ss(s_tm, desc_from_lo(q_lo + off), desc_from_lo(ka + off), idesc_qk,
                                 k > 0 ? 1u : 0u);
                 }
                 ptx::mma_commit(bar(L::bSFull + i));

@@ -149,11 +149,6 @@ __device__ __forceinline__ void reg_dealloc() {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 
-// Named barrier over `count` threads (a multiple of 32).
-__device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t count) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
-}
-
 // ---------------------------------------------------------------- tcgen05
 // Tensor Memory allocation: one warp allocates `ncols` columns (power of two,
 // >= 32) and the hardware writes the base address to shared memory at `dst`.
@@ -188,16 +183,6 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-
-// D(tmem) (+)= A(tmem) * B(smem desc), kind::f16.
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
 // Arrive once on `bar` when every tcgen05 async operation this thread issued
@@ -235,16 +220,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32
         "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
         "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
         "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-        "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-        "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
-        "r"(r[15])
         : "memory");
 }
 
@@ -295,12 +270,6 @@ __device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
     return d;
 }
 
-__device__ __forceinline__ uint64_t f2_sub(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("sub.rn.ftz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-
 __device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
     uint64_t d;
     asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
@@ -315,13 +284,6 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
     return r;
 }
 
-// bf16x2 word from a packed FP32 pair (low lane -> bits [0,16)).
-__device__ __forceinline__ uint32_t pack_bf16x2_from(uint64_t v) {
-    float lo, hi;
-    f2_unpack(v, lo, hi);
-    return pack_bf16x2(lo, hi);
-}
-
 }  // namespace ptx
 
 // ---------------------------------------------------------------- descriptors
@@ -330,18 +292,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2_from(uint64_t v) {
 // [32,46) stride-dimension byte offset >> 4, [46,48) version (1 on sm_100),
 // [49,52) base offset (0: atoms are 1024-byte aligned), [61,64) layout
 // (2 = 128-byte swizzle).
-__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
-                                                    uint32_t sbo_bytes) {
-    uint64_t d = 0;
-    d |= static_cast<uint64_t>((saddr >> 4) & 0x3FFFu);
-    d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-    d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-    d |= static_cast<uint64_t>(1) << 46;
-    d |= static_cast<uint64_t>(2) << 61;
-    return d;
-}
-
-// The same descriptor split in two 32-bit words.  For every operand here the
+// It is kept split in two 32-bit words.  For every operand here the
 // high word is the same (stride offset 1024 bytes, version 1, 128-byte
 // swizzle); the low word carries the start address and the leading offset,
 // so a K step only adds (byte offset >> 4) to it (the 14-bit address field
@@ -358,6 +309,7 @@ __device__ __forceinline__ uint64_t desc_from_lo(uint32_t lo) {
 
 // Instruction descriptor for kind::f16 with BF16 A/B and FP32 D:
 // [4,6) D format (1 = F32), [7,10) A format (1 = BF16), [10,13) B format,
+// bit 13 negate A (kIdescNegateA), bit 14 negate B,
 // bit 15 A major (0 = K-major), bit 16 B major (1 = MN-major),
 // [17,23) N >> 3, [24,29) M >> 4.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, int a_mn_major,
@@ -366,5 +318,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int m, int n, int a_mn_maj
            (static_cast<uint32_t>(b_mn_major) << 16) | (static_cast<uint32_t>(n >> 3) << 17) |
            (static_cast<uint32_t>(m >> 4) << 24);
 }
+constexpr uint32_t kIdescNegateA = 1u << 13;
 
 }  // namespace sdpa10

@@ -77,8 +77,6 @@ def call(lib, q=A, k=A, v=A, o=None, lse=None, b=1, hq=2, hkv=2, sq=256, sk=256,
     (dict(causal=2), attn.ATTN_ERR_INVALID),
     (dict(scale=float("nan")), attn.ATTN_ERR_INVALID),
     (dict(scale=float("inf")), attn.ATTN_ERR_INVALID),
-    (dict(scale=0.0), attn.ATTN_ERR_UNSUPPORTED),
-    (dict(scale=-0.1), attn.ATTN_ERR_UNSUPPORTED),
     (dict(q=A + 8), attn.ATTN_ERR_ALIGN),
     (dict(k=A + 4), attn.ATTN_ERR_ALIGN),
     (dict(v=A + 2), attn.ATTN_ERR_ALIGN),
@@ -101,6 +99,16 @@ def test_error_writes_nothing(lib):
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-device path")
 def test_no_device_reports_cuda_error(lib):
     assert call(lib) == attn.ATTN_ERR_CUDA
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks validation on the no-device path")
+@pytest.mark.parametrize("scale", [0.0, -0.0, -0.1, -3.0, 1e-30, 1e3])
+def test_any_finite_scale_passes_validation(lib, scale):
+    # Every finite scale is a valid argument (the formula has no sign or size
+    # condition on it): validation accepts it and the call then fails only for
+    # want of a device.
+    assert call(lib, scale=scale) == attn.ATTN_ERR_CUDA
+    assert call(lib, scale=scale, causal=1) == attn.ATTN_ERR_CUDA
 
 
 def test_host_workspace_bytes(lib):

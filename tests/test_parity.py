@@ -74,6 +74,36 @@ def test_scales(scale):
     check(q, k, v, True, scale, what=f"scale={scale}")
 
 
+@pytest.mark.parametrize("scale", [-0.09, -1.0, 0.0, -0.0])
+@pytest.mark.parametrize("causal", [False, True])
+def test_negative_and_zero_scale(scale, causal):
+    # The formula puts no condition on the scale.  A negative scale favours
+    # the keys least aligned with the query; scale 0 gives uniform weights
+    # over the visible keys (LSE = ln of their count).
+    q, k, v = make_qkv(2, 4, 2, 300, 700, seed=5100)
+    check(q, k, v, causal, scale, what=f"scale={scale} causal={causal}")
+
+
+def test_rescale_branch_forced():
+    # Keys whose scores beat every earlier key block's maximum by much more
+    # than 2^8 in the exponent force the running output to be rescaled
+    # (twice per row: at key 300 and again at key 450); key 200 raises the
+    # maximum by less than 2^8, which must not rescale.  Every row's result
+    # then depends on the correction being applied exactly: a skipped or
+    # doubled correction weighs the early keys wrong by a factor > 2^16.
+    b, h, s = 1, 2, 512
+    g = torch.Generator().manual_seed(6250)
+    q = (1.0 + 0.1 * torch.randn(b, s, h, 128, generator=g)).to(torch.bfloat16)
+    k = 0.1 * torch.randn(b, s, h, 128, generator=g)
+    k[:, 200] = 0.4   # score ~ 51 * scale -> exponent ~ 6.5 above block 0
+    k[:, 300] = 1.0   # ~ 128 * scale -> ~ 16 above
+    k[:, 450] = 2.0   # ~ 256 * scale -> another ~ 16
+    k = k.to(torch.bfloat16)
+    v = torch.randn(b, s, h, 128, generator=g).to(torch.bfloat16)
+    for causal in (False, True):
+        check(q, k, v, causal, SCALE, what=f"forced rescale causal={causal}")
+
+
 def test_many_tiles_more_than_sms():
     # 2 * 8 * 12 = 192 tiles > 148 SMs: exercises the persistent loop and the
     # reuse of TMEM, barriers and the Q double buffer across tiles.
@@ -182,7 +212,7 @@ def _rows_for(w, n):
     return sample_rows(w.batch, w.h_q, w.seq, n, seed=w.seed + 7919)
 
 
-FULL = ["mha_b8_h16_s4096", "gqa_b8_h16_kv2_s2048", "mqa_b8_h16_kv1_s2048"]
+FULL = ["tiny_b1_h2_s256", "mha_b8_h16_s4096", "gqa_b8_h16_kv2_s2048", "mqa_b8_h16_kv1_s2048"]
 SAMPLED = ["mha_b4_h16_s8192", "mha_b2_h16_s16384", "mha_b1_h16_s32768_k3"]
 
 
@@ -190,11 +220,11 @@ SAMPLED = ["mha_b4_h16_s8192", "mha_b2_h16_s16384", "mha_b1_h16_s32768_k3"]
 @pytest.mark.parametrize("causal", [False, True])
 def test_workload_configs(name, causal):
     """Every config at full size, in the launch configuration the bench
-    times; the oracle evaluates 512 sampled query rows per head on the long
-    sequences and 256 per head on the others (always including rows 0, 1,
-    127, 128, 255, 256 and s-1)."""
+    times.  The oracle evaluates every query row of the 256-, 2K- and
+    4K-sequence configs, and 512 sampled query rows per head of the 8K-32K
+    ones (always including rows 0, 1, 127, 128, 255, 256 and s-1)."""
     w = WORKLOADS[name]
     q, k, v = workload_qkv(w)
-    rows = _rows_for(w, 512 if w.sampled else 256)
+    rows = _rows_for(w, 512) if w.sampled else None
     m = check(q, k, v, causal, w.scale, rows=rows, what=f"{name} causal={causal}")
     print(name, causal, m)
