@@ -90,6 +90,38 @@ def _stream_handle(stream) -> int | None:
     return stream.cuda_stream
 
 
+def _stream_obj(stream, device):
+    """The torch stream object the kernels of a call run on."""
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream(device)
+    if isinstance(stream, int):
+        return torch.cuda.ExternalStream(stream, device=device)
+    return stream
+
+
+def _alloc_on(stream, device, fn):
+    """Allocate with ``fn()`` on the launch stream, so the caching allocator
+    never hands a buffer that a kernel of this call still uses to work queued
+    on another stream once the buffer is dropped."""
+    import torch
+    with torch.cuda.stream(_stream_obj(stream, device)):
+        return fn()
+
+
+def _check_out(t, name, shape, dtype, device):
+    """A caller-supplied output must match what the kernel writes: the C side
+    can check only null and alignment."""
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}")
+
+
 def _check_qkv(q, k, v):
     import torch
     for name, t in (("q", q), ("k", k), ("v", v)):
@@ -106,6 +138,22 @@ def _check_qkv(q, k, v):
     return b, s_q, h_q, h_kv, s_k, d
 
 
+def _outputs(q, o, lse, o_shape, lse_shape, stream, o_dtype=None):
+    """Check caller-supplied outputs, or allocate them on the launch stream."""
+    import torch
+    o_dtype = o_dtype or torch.bfloat16
+    if o is None:
+        o = _alloc_on(stream, q.device, lambda: torch.empty(o_shape, dtype=o_dtype, device=q.device))
+    else:
+        _check_out(o, "o", o_shape, o_dtype, q.device)
+    if lse is None:
+        lse = _alloc_on(stream, q.device,
+                        lambda: torch.empty(lse_shape, dtype=torch.float32, device=q.device))
+    else:
+        _check_out(lse, "lse", lse_shape, torch.float32, q.device)
+    return o, lse
+
+
 def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, lse=None,
              stream=None):
     """O, LSE = attention forward on CUDA tensors [batch, seq, heads, 128] (BF16).
@@ -120,10 +168,7 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, 
             raise ValueError(f"{name} must be a CUDA tensor")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if o is None:
-        o = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
+    o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
     rc = load_library().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                  lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d, int(bool(causal)),
                                  float(scale), _stream_handle(stream))
@@ -156,13 +201,15 @@ def attn_fwd_split(q, k, v, causal: bool = False, scale: float | None = None,
         scale = 1.0 / math.sqrt(d)
     if n_splits is None:
         n_splits = max(1, num_splits(b, h_q, h_kv, s_q, s_k, causal, d))
-    if o is None:
-        o = torch.empty_like(q)
-    if lse is None:
-        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
+    o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
     if workspace is None:
-        workspace = torch.empty(split_workspace_bytes(b, h_q, s_q, n_splits), dtype=torch.uint8,
-                                device=q.device)
+        # Dropped on return while the two kernels may still run: allocated on
+        # their stream, so its memory is not reused before they finish.
+        nbytes = split_workspace_bytes(b, h_q, s_q, n_splits)
+        workspace = _alloc_on(stream, q.device,
+                              lambda: torch.empty(nbytes, dtype=torch.uint8, device=q.device))
+    elif workspace.device != q.device or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on the inputs' device")
     rc = load_library().attn_fwd_split(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                        lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
                                        int(bool(causal)), float(scale), int(n_splits),
@@ -185,10 +232,8 @@ def attn_fwd_partials(q, k, v, causal: bool = False, scale: float | None = None,
             raise ValueError(f"{name} must be a CUDA tensor")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if o_part is None:
-        o_part = torch.empty((b, h_q, s_q, d), dtype=torch.float32, device=q.device)
-    if lse_part is None:
-        lse_part = torch.empty((b, h_q, s_q), dtype=torch.float32, device=q.device)
+    o_part, lse_part = _outputs(q, o_part, lse_part, (b, h_q, s_q, d), (b, h_q, s_q), stream,
+                                o_dtype=torch.float32)
     rc = load_library().attn_fwd_partials(q.data_ptr(), k.data_ptr(), v.data_ptr(),
                                           o_part.data_ptr(), lse_part.data_ptr(), b, h_q, h_kv,
                                           s_q, s_k, d, int(bool(causal)), float(scale),
@@ -211,10 +256,9 @@ def merge_partials(o_parts, lse_parts, o=None, lse=None, stream=None):
     n, b, h_q, s_q, d = o_parts.shape
     if tuple(lse_parts.shape) != (n, b, h_q, s_q):
         raise ValueError("o_parts and lse_parts shapes disagree")
-    if o is None:
-        o = torch.empty((b, s_q, h_q, d), dtype=torch.bfloat16, device=o_parts.device)
-    if lse is None:
-        lse = torch.empty((b, h_q, s_q), dtype=torch.float32, device=o_parts.device)
+    if not o_parts.is_cuda or lse_parts.device != o_parts.device:
+        raise ValueError("partials must be CUDA tensors on one device")
+    o, lse = _outputs(o_parts, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
     rc = load_library().attn_merge_partials(o_parts.data_ptr(), lse_parts.data_ptr(), n, b, h_q,
                                             s_q, d, o.data_ptr(), lse.data_ptr(),
                                             _stream_handle(stream))
@@ -239,9 +283,14 @@ def attn_fwd_host(q, k, v, o, lse, workspace, causal: bool = False, scale: float
     """Forward on HOST tensors (pinned for asynchronous copies) through the
     C entry point that copies in, runs and copies out.  ``workspace`` is a
     CUDA uint8 tensor of at least :func:`host_workspace_bytes` bytes."""
+    import torch
     b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
+    _check_out(o, "o", (b, s_q, h_q, d), torch.bfloat16, q.device)
+    _check_out(lse, "lse", (b, h_q, s_q), torch.float32, q.device)
+    if not workspace.is_cuda or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous CUDA tensor")
     rc = load_library().attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                       lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
                                       int(bool(causal)), float(scale), workspace.data_ptr(),

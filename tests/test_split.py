@@ -165,3 +165,41 @@ def test_partials_of_key_shards_merge_to_the_whole():
     got_l = parts[1][1].cpu()[bi, hi_, r].double().numpy()
     assert np.max(np.abs(got_o - o_r)) < 2e-3  # FP32 partial: no BF16 rounding of O
     assert np.max(np.abs(got_l - l_r)) < 1e-3
+
+
+def test_split_on_side_stream_keeps_its_workspace():
+    # The binding allocates the partials workspace itself and drops it on
+    # return while the kernels run on a side stream; a same-sized buffer
+    # allocated and filled on the default stream right after must not share
+    # its memory (else the fill corrupts the partials).
+    b, hq, sq, sk, n = 1, 16, 256, 32768, 8
+    q, k, v = make_qkv(b, hq, hq, sq, sk, seed=7600)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    want, want_lse = run_split(q, k, v, False, n)
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    for _ in range(5):
+        o, lse = attn.attn_fwd_split(qd, kd, vd, scale=SCALE, n_splits=n, stream=side)
+        junk = torch.empty(attn.split_workspace_bytes(b, hq, sq, n), dtype=torch.uint8,
+                           device="cuda")
+        junk.fill_(0xFF)  # NaN patterns if it aliased the partials
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        assert torch.equal(o, want) and torch.equal(lse, want_lse)
+    assert attn.attn_status() == attn.ATTN_OK
+
+
+def test_binding_checks_output_tensors():
+    q, k, v = make_qkv(1, 2, 2, 256, 256, seed=7700)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    with pytest.raises(ValueError):
+        attn.attn_fwd(qd, kd, vd, o=torch.empty(1, 128, 2, 128, dtype=torch.bfloat16,
+                                                device="cuda"))
+    with pytest.raises(TypeError):
+        attn.attn_fwd(qd, kd, vd, lse=torch.empty(1, 2, 256, dtype=torch.float16, device="cuda"))
+    with pytest.raises(ValueError):
+        attn.attn_fwd_partials(qd, kd, vd, o_part=torch.empty(1, 2, 255, 128, device="cuda"))
+    with pytest.raises(ValueError):
+        attn.attn_fwd_split(qd, kd, vd, n_splits=2,
+                            lse=torch.empty(1, 256, 2, dtype=torch.float32,
+                                            device="cuda").transpose(1, 2))
