@@ -2,11 +2,15 @@
 """Throughput of the fused attention forward on B200.
 
 One step = the whole hot path over one batch: a non-causal and a causal
-forward of the MHA workload (batch 8, 16 heads, sequence 4096, head dim 128,
-BF16), inputs resident in HBM.  The metric is attention-forward TFLOPS,
-counting 4*b*h*s_q*s_k*d FLOPs per forward, halved for the causal one.
+forward of the largest single-GPU workload (batch 1, 16 heads, sequence
+32768, head dim 128, BF16, K drawn x3), inputs resident in HBM.  The metric
+is attention-forward TFLOPS, counting 4*b*h*s_q*s_k*d FLOPs per forward,
+halved for the causal one.  The same line carries a per-configuration block:
+every workload, both masks, each launch timed alone with CUDA events after
+an L2 flush.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--no-configs]
 
 Prints one JSON line (rank 0).  Multi-GPU runs (torchrun) are replicas: each
 rank runs its own batch (weak scaling), timed on the device, max over ranks.
@@ -44,7 +48,14 @@ def parse_args():
     ap.add_argument("--steps", type=int, default=400)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--workload", default="mha_b8_h16_s4096", choices=sorted(WORKLOADS))
+    ap.add_argument("--workload", default="mha_b1_h16_s32768_k3", choices=sorted(WORKLOADS))
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the per-configuration timing block")
+    ap.add_argument("--config-launches", type=int, default=20,
+                    help="timed launches per (configuration, mask) in that block")
+    ap.add_argument("--only", choices=["configs", "split"],
+                    help="run only the per-configuration block or only the split-KV cases "
+                         "(for profiling) and print them as one JSON line")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
@@ -191,38 +202,51 @@ def whole_job_tflops(world: int, flops_per_step: float, steps: int, max_ms: floa
 
 
 # ------------------------------------------------------------------ oracle arm
-def oracle_sample_rate(w, target_s: float, seed_offset: int = 0):
-    """Time the FP64 oracle on a bounded row sample of the workload (both
-    masks).  Returns (TFLOPS in the metric's convention, seconds, rows/head,
-    threads)."""
+def _head_slices(w, q, k, v, i):
+    """The i-th (batch, query head) of the workload, cycling through all of
+    them: the slices of Q, K and V that head reads."""
+    group = w.h_q // w.h_kv
+    bi, hi = i % w.batch, (i // w.batch) % w.h_q
+    gi = hi // group
+    return (q[bi:bi + 1, :, hi:hi + 1].contiguous(), k[bi:bi + 1, :, gi:gi + 1].contiguous(),
+            v[bi:bi + 1, :, gi:gi + 1].contiguous())
+
+
+def _oracle_step(w, qs, ks, vs, n_rows, seed):
+    """The FP64 oracle on n_rows seeded rows of one head, both masks.
+    Returns (FLOPs in the metric's convention, seconds)."""
+    import oracle
+    d = 128
+    rows = sample_rows(1, 1, w.seq, n_rows, seed=seed, include_edges=False)
+    t0 = time.perf_counter()
+    f = 0.0
+    for causal in MODES:
+        oracle.attn_fwd(qs, ks, vs, causal, w.scale, rows=rows)
+        f += float(4 * d * ((rows.astype("int64") + 1).sum() if causal else w.seq * rows.size))
+    return f, time.perf_counter() - t0
+
+
+def oracle_sample_rate(w, target_s: float):
+    """Time the FP64 oracle on a bounded sample of the workload: per step one
+    (batch, query head) slice (so decoding inputs the sample never reads is
+    not counted as oracle time) and a seeded row sample of it, both masks,
+    steps repeated until about target_s seconds.  Returns (TFLOPS in the
+    metric's convention, seconds, rows per step, steps, threads)."""
     import oracle
     q, k, v = workload_qkv(w)
-    d = 128
-
-    def flops(rows, causal):
-        if causal:
-            return float(4 * d * (rows.astype("int64") + 1).sum())
-        return float(4 * d * w.seq * rows.size)
-
-    def run(n_rows, seed):
-        rows = sample_rows(w.batch, w.h_q, w.seq, n_rows, seed=seed, include_edges=False)
-        t0 = time.perf_counter()
-        f = 0.0
-        for causal in MODES:
-            oracle.attn_fwd(q, k, v, causal, w.scale, rows=rows)
-            f += flops(rows, causal)
-        return f, time.perf_counter() - t0
-
-    # Calibrate t(n) = fixed + per_row * n from two small samples (each call
-    # also pays a fixed cost for decoding the whole inputs), then size the
-    # timed sample to about target_s.
-    _, t1 = run(1, w.seed + 1 + seed_offset)
-    _, t4 = run(4, w.seed + 3 + seed_offset)
-    per_n = max((t4 - t1) / 3.0, 1e-6)
-    fixed = max(t1 - per_n, 0.0)
-    n = max(1, min(w.seq, int((target_s - fixed) / per_n)))
-    f, t = run(n, w.seed + 2 + seed_offset)
-    return f / t / 1e12, t, n, oracle.num_threads()
+    # Size the row sample so one step costs about target_s / 8.
+    qs, ks, vs = _head_slices(w, q, k, v, 0)
+    _, t1 = _oracle_step(w, qs, ks, vs, 8, w.seed + 1)
+    n = max(1, min(w.seq, int(8 * (target_s / 8) / max(t1, 1e-6))))
+    flops = secs = 0.0
+    steps = 0
+    while secs < target_s and steps < 64:
+        qs, ks, vs = _head_slices(w, q, k, v, steps)
+        f, t = _oracle_step(w, qs, ks, vs, n, w.seed + 2 + steps)
+        flops += f
+        secs += t
+        steps += 1
+    return flops / secs / 1e12, secs, n, steps, oracle.num_threads()
 
 
 def run_reference(args, world, rank):
@@ -233,29 +257,13 @@ def run_reference(args, world, rank):
     per_step = budget / max(1, args.steps + args.warmup)
     import oracle
     q, k, v = workload_qkv(w)
-    d = 128
     times, flops_total = [], 0.0
-    rows_n = None
-    group = w.h_q // w.h_kv
+    rows_n = 1
     for i in range(args.warmup + args.steps):
-        if rows_n is None:
-            rows_n = 1
-        # One (batch, query head) of the workload per step, at its full
-        # sequence length: the oracle is handed only the slices that head
-        # reads (so a small row sample does not pay for decoding the whole
-        # batch), and the rows are sampled within it.
-        bi, hi = i % w.batch, (i // w.batch) % w.h_q
-        gi = hi // group
-        qs = q[bi:bi + 1, :, hi:hi + 1].contiguous()
-        ks = k[bi:bi + 1, :, gi:gi + 1].contiguous()
-        vs = v[bi:bi + 1, :, gi:gi + 1].contiguous()
-        rows = sample_rows(1, 1, w.seq, rows_n, seed=w.seed + 100 + i, include_edges=False)
-        t0 = time.perf_counter()
-        f = 0.0
-        for causal in MODES:
-            oracle.attn_fwd(qs, ks, vs, causal, w.scale, rows=rows)
-            f += float(4 * d * ((rows.astype("int64") + 1).sum() if causal else w.seq * rows.size))
-        dt = time.perf_counter() - t0
+        # One (batch, query head) of the workload per step at its full
+        # sequence length, on a seeded row sample sized in the warm-up.
+        qs, ks, vs = _head_slices(w, q, k, v, i)
+        f, dt = _oracle_step(w, qs, ks, vs, rows_n, w.seed + 100 + i)
         if i < args.warmup:
             # size the sample so one step costs about `per_step` seconds
             rows_n = max(1, min(w.seq, int(rows_n * per_step / max(dt, 1e-6))))
@@ -359,7 +367,8 @@ def run_ours(args, world, rank, local):
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
         "warmup": args.warmup, "ms_per_step": total_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-        "data": "synthetic (seeded N(0,1) BF16; inputs 402 MB > 126 MB L2, no flush needed)",
+        "data": f"synthetic (seeded N(0,1) BF16; inputs {w.input_bytes() / 1e6:.0f} MB > 126 MB "
+                "L2, no flush needed)",
         "config": {"workload": w.name, "batch": w.batch, "h_q": w.h_q, "h_kv": w.h_kv,
                    "seq": w.seq, "head_dim": 128, "modes": ["noncausal", "causal"],
                    "l2": "inputs larger than L2", "parallelism": f"replicas x{world}"},
@@ -373,14 +382,133 @@ def run_ours(args, world, rank, local):
 
     if not args.no_e2e:
         line["e2e"] = run_e2e(args, w, q, k, v, world)
+    if world == 1 and not args.no_configs:
+        line["configs"] = run_configs(args, peaks)
+        line["configs"]["split_kv"] = run_split_cases(args, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tfl, secs, n, cores = oracle_sample_rate(w, args.cpu_seconds)
+        tfl, secs, n, steps, cores = oracle_sample_rate(w, args.cpu_seconds)
         line["cpu_baseline"] = {
             "value": tfl, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{n} seeded query rows per (batch, head) of {w.name}, both masks, "
-                      f"{secs:.1f} s; FLOPs counted as 4*d*visible keys per row"}
+            "sample": f"{steps} (batch, head) slices of {w.name}, {n} seeded query rows each, "
+                      f"both masks, {secs:.1f} s; FLOPs counted as 4*d*visible keys per row"}
     if rank == 0:
         print(json.dumps(line), flush=True)
+
+
+def run_configs(args, peaks):
+    """Every workload, both masks: each launch timed alone with CUDA events on
+    the launching stream after a 256 MB L2 flush (so the small workloads are
+    not measured from a warm L2).  Median over the timed launches."""
+    from scaled_dot_product_10_b200 import attn
+    peak = float(peaks["bf16_tflops"])
+    hbm = float(peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"]))
+    stream = torch.cuda.current_stream()
+    sh = stream.cuda_stream
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    out = {}
+    for name, w in WORKLOADS.items():
+        q, k, v = (t.cuda() for t in workload_qkv(w))
+        o = torch.empty_like(q)
+        lse = torch.empty((w.batch, w.h_q, w.seq), dtype=torch.float32, device="cuda")
+        ptrs = (q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr())
+        entry = {}
+        for causal in MODES:
+            def launch():
+                rc = attn.attn_fwd_raw(*ptrs, w.batch, w.h_q, w.h_kv, w.seq, w.seq, 128, causal,
+                                       w.scale, sh)
+                if rc != attn.ATTN_OK:
+                    raise attn.AttnError(rc, "attn_fwd")
+            for _ in range(3):
+                launch()
+            times = []
+            for _ in range(args.config_launches):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                launch()
+                b.record(stream)
+                times.append((a, b))
+            torch.cuda.synchronize()
+            ms = statistics.median(a.elapsed_time(b) for a, b in times)
+            tf = w.flops(causal) / (ms * 1e-3) / 1e12
+            gbs = w.algorithmic_bytes() / (ms * 1e-3) / 1e9
+            entry["causal" if causal else "noncausal"] = {
+                "ms_per_launch": ms, "tflops": tf, "frac": tf / peak,
+                "frac_of_spec_2250": tf / SPEC_PEAK_TFLOPS, "alg_gbs": gbs,
+                "hbm_frac": gbs / hbm}
+        rc = attn.attn_status()
+        if rc != attn.ATTN_OK:
+            raise attn.AttnError(rc, f"kernel status after {name}")
+        out[name] = entry
+        del q, k, v, o, lse
+    del flush
+    torch.cuda.empty_cache()
+    return {"timing": f"median of {args.config_launches} launches per mask, each after a "
+                      "256 MB L2 flush; CUDA events on the launching stream",
+            "frac_of": "measured bf16 burst peak", "workloads": out}
+
+
+# Few query rows over long key sequences: where the pairs of one launch leave
+# SMs idle and the split-KV forward pays off.
+# (name, batch, h_q, h_kv, s_q, s_k, seed); non-causal, N(0,1) BF16.
+SPLIT_CASES = [
+    ("few_q_b1_h16_q256_k32768", 1, 16, 16, 256, 32768, 1101),
+    ("few_q_b1_h16_q512_k32768", 1, 16, 16, 512, 32768, 1102),
+    ("few_q_b2_h16_q128_k16384", 2, 16, 16, 128, 16384, 1103),
+    ("few_q_gqa_b1_h32_kv4_q256_k65536", 1, 32, 4, 256, 65536, 1104),
+]
+
+
+def run_split_cases(args, peaks):
+    """attn_fwd against attn_fwd_split (the library's range count; forward
+    plus merge) on the few-query cases, each launch timed alone after an L2
+    flush, median of the timed launches."""
+    from scaled_dot_product_10_b200 import attn
+    from scaled_dot_product_10_b200.workloads import make_qkv
+    peak = float(peaks["bf16_tflops"])
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    def timed(f):
+        for _ in range(3):
+            f()
+        ev = []
+        for _ in range(args.config_launches):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            f()
+            b.record(stream)
+            ev.append((a, b))
+        torch.cuda.synchronize()
+        return statistics.median(a.elapsed_time(b) for a, b in ev)
+
+    out = {}
+    for name, b, hq, hkv, sq, sk, seed in SPLIT_CASES:
+        q, k, v = (t.cuda() for t in make_qkv(b, hq, hkv, sq, sk, seed=seed))
+        scale = 1.0 / math.sqrt(128)
+        o = torch.empty_like(q)
+        lse = torch.empty((b, hq, sq), dtype=torch.float32, device="cuda")
+        n = attn.num_splits(b, hq, hkv, sq, sk)
+        ws = torch.empty(attn.split_workspace_bytes(b, hq, sq, n), dtype=torch.uint8,
+                         device="cuda")
+        t_plain = timed(lambda: attn.attn_fwd(q, k, v, scale=scale, o=o, lse=lse))
+        t_split = timed(lambda: attn.attn_fwd_split(q, k, v, scale=scale, n_splits=n, o=o,
+                                                    lse=lse, workspace=ws))
+        rc = attn.attn_status()
+        if rc != attn.ATTN_OK:
+            raise attn.AttnError(rc, f"kernel status after {name}")
+        flops = 4.0 * b * hq * sq * sk * 128
+        byts = 2 * (b * sq * hq * 128 * 2) + 2 * (b * sk * hkv * 128 * 2) + b * hq * sq * 4
+        out[name] = {"n_splits": n, "ms_attn_fwd": t_plain, "ms_split": t_split,
+                     "tflops_attn_fwd": flops / (t_plain * 1e-3) / 1e12,
+                     "tflops_split": flops / (t_split * 1e-3) / 1e12,
+                     "frac_split": flops / (t_split * 1e-3) / 1e12 / peak,
+                     "speedup": t_plain / t_split,
+                     "alg_gbs_split": byts / (t_split * 1e-3) / 1e9}
+    return out
 
 
 def run_e2e(args, w, q, k, v, world):
@@ -425,6 +553,13 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         return run_reference(args, world, rank)
     world, rank, local = dist_setup(args)
+    if args.only:
+        from scaled_dot_product_10_b200 import attn
+        attn.load_library()
+        peaks, _ = load_peaks()
+        part = run_configs(args, peaks) if args.only == "configs" else run_split_cases(args, peaks)
+        print(json.dumps({"only": args.only, args.only: part}), flush=True)
+        return 0
     try:
         run_ours(args, world, rank, local)
     finally:

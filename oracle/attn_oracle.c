@@ -18,20 +18,23 @@
  *        causal: S[i][j] = -inf for j > i + (s_k - s_q)    (mask; the
  *        intelliparadigm.com AVO page, section 2.2, fuses the mask into
  *        the softmax -- here it is simply applied to S.  The pages only
- *        use s_q = s_k, where this is j > i; for s_q < s_k the mask is
- *        aligned to the bottom-right corner, so the last query sees every
- *        key -- the reading stated in the design notes)
+ *        use s_q = s_k, where this is j > i.  They never say how the mask
+ *        lines up when s_q < s_k; the reading taken here aligns it to the
+ *        bottom-right corner: the s_q queries are taken to be the LAST s_q
+ *        positions of the key sequence, so the last query sees every key
+ *        and s_q > s_k is refused, since a row would then see no key)
  *        sliding window (window_left >= 0, causal only): also
  *        S[i][j] = -inf for j < i + (s_k - s_q) - window_left, so row i
- *        sees the window_left + 1 keys ending at its diagonal (the local
- *        window variant; the reading is stated in the design notes)
+ *        sees the window_left + 1 keys ending at its diagonal.  The pages
+ *        name a local-window variant without defining it; the reading
+ *        taken is this one-sided window on top of the causal mask)
  *     2. m_i = max_j S[i][j];  E = exp(S - m_i);  l_i = sum_j E[i][j];
  *        P = E / l_i        (numerically stable softmax with the scale
  *        applied before the max, as in the AVO page, section 3.1 item 2)
  *     3. O[i][:] = sum_j P[i][j] V[j][:]
  *   plus the per-row log-sum-exp of the scaled scores, LSE_i = m_i + ln l_i
- *   (natural log; not on the pages -- the reading is stated in the design
- *   notes).
+ *   (the pages do not define it; the reading taken is the natural log of
+ *   the sum of exp over the scaled, masked scores of the row, m included).
  *
  *   Head sharing (grouped-query attention, rkmt.cn page section 3.2): query
  *   head h reads key/value head h / (h_q / h_kv) -- contiguous groups.

@@ -43,6 +43,10 @@ class Workload:
         f = 4.0 * self.batch * self.h_q * self.seq * self.seq * HEAD_DIM
         return f / 2 if causal else f
 
+    def input_bytes(self) -> int:
+        """Q, K and V (BF16)."""
+        return 2 * HEAD_DIM * (self.batch * self.seq * self.h_q + 2 * self.batch * self.seq * self.h_kv)
+
     def algorithmic_bytes(self) -> int:
         """Q, K, V and O moved once (BF16) plus the FP32 LSE."""
         q = self.batch * self.seq * self.h_q * HEAD_DIM * 2
