@@ -113,3 +113,45 @@ def attn_fwd(q, k, v, causal: bool, scale: float, rows=None, want_p: bool = Fals
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (code {rc})")
     return o, lse, p
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal: bool, scale: float,
+                    window_left: int = -1, lib=None):
+    """Packed variable-length batch: the definition applied to each sequence
+    on its own (attention never crosses sequences).
+
+    q: [total_q, h_q, d] bf16; k, v: [total_k, h_kv, d].  Sequence b holds
+    query rows cu_seqlens_q[b] .. cu_seqlens_q[b+1] - 1 and keys
+    cu_seqlens_k[b] .. cu_seqlens_k[b+1] - 1; the causal mask (and window)
+    is that of a single problem with that sequence's s_q and s_k.  A
+    sequence with no query rows contributes nothing; one with query rows but
+    no keys is rejected.
+
+    Returns (o [total_q, h_q, d] float64, lse [h_q, total_q] float64).
+    """
+    qb, kb, vb = _as_bits(q), _as_bits(k), _as_bits(v)
+    cu_q = [int(x) for x in np.asarray(cu_seqlens_q).reshape(-1)]
+    cu_k = [int(x) for x in np.asarray(cu_seqlens_k).reshape(-1)]
+    if len(cu_q) != len(cu_k) or len(cu_q) < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k need batch + 1 entries each")
+    total_q, h_q, d = qb.shape
+    total_k, h_kv, dk = kb.shape
+    if vb.shape != kb.shape or dk != d:
+        raise ValueError("shape mismatch between q, k and v")
+    if cu_q[0] != 0 or cu_k[0] != 0 or cu_q[-1] != total_q or cu_k[-1] != total_k:
+        raise ValueError("cu_seqlens must start at 0 and end at the packed lengths")
+    o = np.zeros((total_q, h_q, d), dtype=np.float64)
+    lse = np.zeros((h_q, total_q), dtype=np.float64)
+    for b in range(len(cu_q) - 1):
+        q0, q1, k0, k1 = cu_q[b], cu_q[b + 1], cu_k[b], cu_k[b + 1]
+        if q1 < q0 or k1 < k0:
+            raise ValueError("cu_seqlens must not decrease")
+        if q1 == q0:
+            continue
+        if k1 == k0:
+            raise ValueError(f"sequence {b} has query rows but no keys")
+        ob, lb, _ = attn_fwd(qb[None, q0:q1], kb[None, k0:k1], vb[None, k0:k1], causal, scale,
+                             lib=lib, window_left=window_left)
+        o[q0:q1] = ob[0].transpose(1, 0, 2)
+        lse[:, q0:q1] = lb[0]
+    return o, lse

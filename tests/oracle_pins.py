@@ -316,6 +316,62 @@ def pin_row_subset(lib):
             assert np.array_equal(ls[0, hi], lf[0, hi, rows[0, hi]])
 
 
+
+
+def _varlen_case(seed, lens_q, lens_k, h_q=4, h_kv=2, d=16):
+    """Packed q [total_q, h_q, d], k/v [total_k, h_kv, d] and cu_seqlens."""
+    cu_q = np.concatenate([[0], np.cumsum(lens_q)]).astype(np.int32)
+    cu_k = np.concatenate([[0], np.cumsum(lens_k)]).astype(np.int32)
+    q, k, v = make_qkv(1, h_q, h_kv, int(cu_q[-1]), int(cu_k[-1]), seed=seed, d=d)
+    return q[0], k[0], v[0], cu_q, cu_k
+
+
+def pin_varlen_matches_block_diagonal_sdpa(lib):
+    """A packed batch equals ONE attention over all packed tokens whose mask
+    forbids every (query, key) pair of different sequences (and, causal,
+    keys past the row's own diagonal in its sequence): torch's float64 SDPA
+    with that explicit boolean mask, and torch.logsumexp of the masked
+    scores."""
+    lens_q, lens_k = [5, 1, 9, 3], [7, 4, 9, 3]
+    q, k, v, cu_q, cu_k = _varlen_case(31, lens_q, lens_k)
+    h_q, h_kv = q.shape[1], k.shape[1]
+    seq_q = np.repeat(np.arange(4), lens_q)
+    seq_k = np.repeat(np.arange(4), lens_k)
+    pos_q = np.arange(cu_q[-1]) - cu_q[seq_q]
+    pos_k = np.arange(cu_k[-1]) - cu_k[seq_k]
+    off = (np.asarray(lens_k) - np.asarray(lens_q))[seq_q]
+    for causal in (False, True):
+        allow = seq_q[:, None] == seq_k[None, :]
+        if causal:
+            allow &= pos_k[None, :] <= (pos_q + off)[:, None]
+        mask = torch.from_numpy(allow)
+        qt = q.double().permute(1, 0, 2)[None]                    # [1, h_q, Tq, d]
+        kt = k.double().permute(1, 0, 2).repeat_interleave(h_q // h_kv, 0)[None]
+        vt = v.double().permute(1, 0, 2).repeat_interleave(h_q // h_kv, 0)[None]
+        want = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask,
+                                                                scale=0.3)
+        scores = (qt @ kt.transpose(-1, -2)) * 0.3
+        want_lse = torch.logsumexp(scores.masked_fill(~mask, float("-inf")), dim=-1)
+        o, lse = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, causal, 0.3, lib=lib)
+        assert np.max(np.abs(o - want[0].permute(1, 0, 2).numpy())) < 1e-10, "varlen O"
+        assert np.max(np.abs(lse - want_lse[0].numpy())) < 1e-10, "varlen LSE"
+
+
+def pin_varlen_sequences_are_independent(lib):
+    """Changing one sequence's tokens changes no other sequence's result."""
+    q, k, v, cu_q, cu_k = _varlen_case(32, [6, 4, 8], [6, 10, 8])
+    o1, l1 = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, False, 0.25, lib=lib)
+    k2, v2 = k.clone(), v.clone()
+    k2[cu_k[1]:cu_k[2]] = bf16(np.full(k2[cu_k[1]:cu_k[2]].shape, 1.5))
+    v2[cu_k[1]:cu_k[2]] = bf16(np.full(v2[cu_k[1]:cu_k[2]].shape, -0.5))
+    o2, l2 = oracle.attn_fwd_varlen(q, k2, v2, cu_q, cu_k, False, 0.25, lib=lib)
+    other = np.r_[cu_q[0]:cu_q[1], cu_q[2]:cu_q[3]]
+    assert np.array_equal(o1[other], o2[other]) and np.array_equal(l1[:, other], l2[:, other])
+    # Identical V rows in the changed sequence: its outputs are -0.5 (the
+    # weights sum to 1 up to FP64 rounding).
+    assert np.all(np.abs(o2[cu_q[1]:cu_q[2]] + 0.5) < 1e-14)
+
+
 ALL_PINS = [
     pin_rows_sum_to_one, pin_identical_v_rows, pin_zero_query, pin_causal_row0,
     pin_causal_rectangular_is_square_suffix, pin_causal_single_query_sees_every_key,
@@ -323,6 +379,7 @@ ALL_PINS = [
     pin_window_row_is_attention_over_its_keys, pin_key_split_merge,
     pin_key_shift, pin_value_affine, pin_key_permutation, pin_gqa_equals_repeated_mha,
     pin_torch_sdpa_f64, pin_golden_closed_forms, pin_row_subset,
+    pin_varlen_matches_block_diagonal_sdpa, pin_varlen_sequences_are_independent,
 ]
 
 
