@@ -82,6 +82,24 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int causal, float scale, void* stream);
 
 /*
+ * attn_fwd_window -- causal attention with a sliding window (the local
+ * window variant of the bjdmk.com.cn survey page, section 2.1): query row i
+ * sees keys i + (s_k - s_q) - window_left .. i + (s_k - s_q), the
+ * window_left keys before its diagonal and the diagonal key itself.
+ * Arguments, layouts and errors as attn_fwd with causal = 1, plus:
+ *
+ *   window_left  >= 0 (ATTN_ERR_INVALID otherwise); 0 leaves each row only
+ *                its diagonal key; >= s_k is the plain causal mask
+ *
+ * Key blocks wholly outside a query block's window are skipped, so the work
+ * grows with window_left, not with s_k.  One launch; asynchronous; allocates
+ * nothing.
+ */
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int batch, int h_q, int h_kv, int s_q, int s_k, int d,
+                    int window_left, float scale, void* stream);
+
+/*
  * attn_fwd_host -- the same forward on HOST buffers: copies q, k, v to the
  * device (cudaMemcpyAsync on `stream`), runs attn_fwd, copies o and lse back,
  * and returns without synchronising (the caller synchronises `stream` before
@@ -192,11 +210,38 @@ int attn_fwd_split(const void* q, const void* k, const void* v, void* o, float* 
  *   lse_part  device, fp32 [batch, h_q, s_q] (written): natural-log
  *             log-sum-exp of the range's scaled scores
  *
+ * With causal = 1 the mask is attn_fwd's, aligned to the bottom-right corner
+ * of THIS call's keys (s_q <= s_k); a shard of a longer key sequence whose
+ * keys do not end at the diagonal needs attn_fwd_partials_shard.
+ *
  * One launch; asynchronous; allocates nothing.
  */
 int attn_fwd_partials(const void* q, const void* k, const void* v, float* o_part,
                       float* lse_part, int batch, int h_q, int h_kv, int s_q, int s_k, int d,
                       int causal, float scale, void* stream);
+
+/*
+ * attn_fwd_partials_shard -- attn_fwd_partials for a key shard that need not
+ * end at the causal diagonal of the whole problem: what one rank of a
+ * key-sequence (context-parallel) split computes when the rank holds keys
+ * [k0, k0 + s_k) of S_k keys in all.  Arguments, layouts and errors as
+ * attn_fwd_partials, plus:
+ *
+ *   diag_offset  causal = 1: query row i sees key j of this call iff
+ *                j <= i + diag_offset.  With the queries as the last s_q of
+ *                the whole key sequence (the bottom-right mask of attn_fwd),
+ *                a shard at global key k0 takes diag_offset = S_k - s_q - k0.
+ *                Negative and large values are allowed (|diag_offset| <=
+ *                2^30); ignored when causal = 0.  s_q > s_k is allowed.
+ *
+ * A row that sees none of the shard's keys gets O_r = 0 and LSE_r = -inf (no
+ * weight in attn_merge_partials).  One launch, or two when some rows see no
+ * key at all (a fill of those rows, then the forward); asynchronous;
+ * allocates nothing.
+ */
+int attn_fwd_partials_shard(const void* q, const void* k, const void* v, float* o_part,
+                            float* lse_part, int batch, int h_q, int h_kv, int s_q, int s_k,
+                            int d, int causal, int diag_offset, float scale, void* stream);
 
 /*
  * attn_merge_partials -- the merge step alone, for partials computed
@@ -247,7 +292,7 @@ int attn_set_wait_timeout_ns(uint64_t ns);
 int attn_selftest_wait_timeout(uint64_t timeout_ns, void* stream);
 
 /* Number of kernel launches the last forward call made (1; 2 for
- * attn_fwd_split: forward + merge). */
+ * attn_fwd_split: forward + merge; 1 or 2 for attn_fwd_partials_shard). */
 int attn_last_launch_count(void);
 
 #ifdef __cplusplus

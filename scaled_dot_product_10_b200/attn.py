@@ -28,6 +28,7 @@ _P = ctypes.c_void_p
 _I = ctypes.c_int
 _SIGNATURES = [
     ("attn_fwd", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]),
+    ("attn_fwd_window", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]),
     ("attn_fwd_host", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
                            _P, ctypes.c_size_t, _P]),
     ("attn_fwd_host_workspace_bytes", ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
@@ -37,6 +38,8 @@ _SIGNATURES = [
     ("attn_fwd_split_workspace_bytes", ctypes.c_size_t, [_I, _I, _I, _I]),
     ("attn_fwd_split", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _I,
                             _P, ctypes.c_size_t, _P]),
+    ("attn_fwd_partials_shard", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                                     ctypes.c_float, _P]),
     ("attn_merge_partials", _I, [_P, _P, _I, _I, _I, _I, _I, _P, _P, _P]),
     ("attn_fwd_partials", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
                                _P]),
@@ -177,6 +180,26 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, 
     return o, lse
 
 
+def attn_fwd_window(q, k, v, window_left: int, scale: float | None = None, o=None, lse=None,
+                    stream=None):
+    """Causal attention where query row i sees only keys
+    i + s_k - s_q - window_left .. i + s_k - s_q.  Returns (o, lse) as
+    :func:`attn_fwd`."""
+    b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
+    rc = load_library().attn_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                        lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
+                                        int(window_left), float(scale), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_window")
+    return o, lse
+
+
 def num_splits(b, h_q, h_kv, s_q, s_k, causal=False, d=128) -> int:
     """Key-range count the library picks for these sizes on the current device."""
     return int(load_library().attn_fwd_num_splits(b, h_q, h_kv, s_q, s_k, d, int(bool(causal))))
@@ -240,6 +263,40 @@ def attn_fwd_partials(q, k, v, causal: bool = False, scale: float | None = None,
                                           _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_partials")
+    return o_part, lse_part
+
+
+def shard_diag_offset(s_k_total: int, s_q: int, key_offset: int) -> int:
+    """Causal diagonal of a key shard at global key ``key_offset`` when the
+    s_q queries are the last s_q positions of ``s_k_total`` keys."""
+    return int(s_k_total) - int(s_q) - int(key_offset)
+
+
+def attn_fwd_partials_shard(q, k, v, causal: bool = False, scale: float | None = None,
+                            diag_offset: int | None = None, o_part=None, lse_part=None,
+                            stream=None):
+    """The unmerged partial of a key shard (see :func:`attn_fwd_partials`);
+    with ``causal`` query row i sees shard key j iff j <= i + diag_offset
+    (default: s_k - s_q, the whole-problem mask).  Rows that see no key of
+    the shard get O_r = 0 and LSE_r = -inf."""
+    import torch
+    b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if diag_offset is None:
+        diag_offset = s_k - s_q
+    o_part, lse_part = _outputs(q, o_part, lse_part, (b, h_q, s_q, d), (b, h_q, s_q), stream,
+                                o_dtype=torch.float32)
+    rc = load_library().attn_fwd_partials_shard(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                o_part.data_ptr(), lse_part.data_ptr(), b, h_q,
+                                                h_kv, s_q, s_k, d, int(bool(causal)),
+                                                int(diag_offset), float(scale),
+                                                _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_partials_shard")
     return o_part, lse_part
 
 

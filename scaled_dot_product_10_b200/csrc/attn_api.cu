@@ -56,7 +56,10 @@ int init_device(int dev, DeviceState** out) {
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return ATTN_ERR_CUDA;
-        if (cudaFuncSetAttribute(attn_fwd_sm100_kernel,
+        if (cudaFuncSetAttribute(attn_fwd_sm100_kernel<false>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 Layout::kAlloc) != cudaSuccess ||
+            cudaFuncSetAttribute(attn_fwd_sm100_kernel<true>,
                                  cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  Layout::kAlloc) != cudaSuccess)
             return ATTN_ERR_CUDA;
@@ -133,8 +136,9 @@ size_t split_workspace_bytes(int batch, int h_q, int s_q, int n_splits) {
 // The forward launch shared by attn_fwd and attn_fwd_split (arguments
 // already validated).  o_part / lse_part null: O and LSE directly.
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int batch,
-               int h_q, int h_kv, int s_q, int s_k, int causal, float scale, int n_splits,
-               int kb_per_split, float* o_part, float* lse_part, void* stream) {
+               int h_q, int h_kv, int s_q, int s_k, int causal, int causal_offset, float scale,
+               int n_splits, int kb_per_split, float* o_part, float* lse_part, void* stream,
+               int window_left = -1) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
     DeviceState* st = nullptr;
@@ -163,7 +167,7 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.n_qb = (s_q + kBlockM - 1) / kBlockM;
     p.n_kb = (s_k + kBlockN - 1) / kBlockN;
     p.causal = causal;
-    p.causal_offset = s_k - s_q;
+    p.causal_offset = causal_offset;
     p.n_pairs = (p.n_qb + 1) / 2;
     p.n_splits = n_splits;
     p.kb_per_split = kb_per_split;
@@ -171,7 +175,14 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     const size_t unit_bytes = 2ull * s_k * kHeadDim * 2;  // K and V of one (batch, kv head)
     const size_t per_sec = kL2SectionBytes / (unit_bytes ? unit_bytes : 1);
     const int units_total = batch * h_kv;
-    p.units_per_section = static_cast<int>(per_sec < 1 ? 1 : (per_sec > (size_t)units_total ? units_total : per_sec));
+    // Non-causal items are all alike: L2 sections keep the K/V of the units
+    // in flight resident.  Causal items differ in length: one section puts
+    // every item in one longest-first order, which the snake deal evens out
+    // across the CTAs (the CTAs on one head then start their key streams
+    // together and share them through L2).
+    p.units_per_section =
+        causal ? units_total
+               : static_cast<int>(per_sec < 1 ? 1 : (per_sec > (size_t)units_total ? units_total : per_sec));
     p.last_section = (units_total - 1) / p.units_per_section;
     p.last_units = units_total - p.last_section * p.units_per_section;
     p.div_splits = FastDiv::make(static_cast<uint32_t>(n_splits));
@@ -192,8 +203,14 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.timeout_ns = g_timeout_ns;
     p.status = st->status;
 
+    p.window_left = window_left;
+
     const int grid = p.num_tiles < st->num_sms ? p.num_tiles : st->num_sms;
-    attn_fwd_sm100_kernel<<<grid, kThreads, Layout::kAlloc,
+    if (window_left >= 0)
+        attn_fwd_sm100_kernel<true><<<grid, kThreads, Layout::kAlloc,
+                                      static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, to, p);
+    else
+        attn_fwd_sm100_kernel<false><<<grid, kThreads, Layout::kAlloc,
                                        static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, to, p);
     g_last_launches = 1;
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
@@ -240,8 +257,21 @@ extern "C" int attn_fwd(const void* q, const void* k, const void* v, void* o, fl
     const int rc = validate(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale);
     if (rc != ATTN_OK) return rc;
     const int n_kb = (s_k + kBlockN - 1) / kBlockN;
-    return launch_fwd(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, causal, scale, 1, n_kb,
-                      nullptr, nullptr, stream);
+    return launch_fwd(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, causal, s_k - s_q, scale, 1,
+                      n_kb, nullptr, nullptr, stream);
+}
+
+extern "C" int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int batch, int h_q, int h_kv, int s_q, int s_k, int d,
+                               int window_left, float scale, void* stream) {
+    const int rc = validate(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, 1, scale);
+    if (rc != ATTN_OK) return rc;
+    if (window_left < 0) return ATTN_ERR_INVALID;
+    const int n_kb = (s_k + kBlockN - 1) / kBlockN;
+    // A window of s_k keys or more is the plain causal mask.
+    const int w = window_left >= s_k ? -1 : window_left;
+    return launch_fwd(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, 1, s_k - s_q, scale, 1, n_kb,
+                      nullptr, nullptr, stream, w);
 }
 
 extern "C" int attn_fwd_num_splits(int batch, int h_q, int h_kv, int s_q, int s_k, int d,
@@ -287,8 +317,8 @@ extern "C" int attn_fwd_split(const void* q, const void* k, const void* v, void*
                                                round_up(static_cast<size_t>(n_splits) * rows *
                                                             kHeadDim * 4,
                                                         256));
-    rc = launch_fwd(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, causal, scale, n_splits,
-                    kb_per_split, o_part, lse_part, stream);
+    rc = launch_fwd(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, causal, s_k - s_q, scale,
+                    n_splits, kb_per_split, o_part, lse_part, stream);
     if (rc != ATTN_OK) return rc;
     rc = launch_merge(o_part, lse_part, n_splits, batch, h_q, s_q, kb_per_split * kBlockN, s_k,
                       causal, o, lse, stream);
@@ -303,8 +333,57 @@ extern "C" int attn_fwd_partials(const void* q, const void* k, const void* v, fl
                             scale);
     if (rc != ATTN_OK) return rc;
     const int n_kb = (s_k + kBlockN - 1) / kBlockN;
-    return launch_fwd(q, k, v, nullptr, nullptr, batch, h_q, h_kv, s_q, s_k, causal, scale, 1,
-                      n_kb, o_part, lse_part, stream);
+    return launch_fwd(q, k, v, nullptr, nullptr, batch, h_q, h_kv, s_q, s_k, causal, s_k - s_q,
+                      scale, 1, n_kb, o_part, lse_part, stream);
+}
+
+extern "C" int attn_fwd_partials_shard(const void* q, const void* k, const void* v,
+                                       float* o_part, float* lse_part, int batch, int h_q,
+                                       int h_kv, int s_q, int s_k, int d, int causal,
+                                       int diag_offset, float scale, void* stream) {
+    if (!q || !k || !v || !o_part || !lse_part) return ATTN_ERR_INVALID;
+    int rc = validate_sizes(batch, h_q, h_kv, s_q, s_k, d);
+    if (rc != ATTN_OK) return rc;
+    if (!std::isfinite(scale) || (causal != 0 && causal != 1)) return ATTN_ERR_INVALID;
+    // Row + diagonal must stay inside 32-bit arithmetic in the kernel.
+    if (diag_offset < -(1 << 30) || diag_offset > (1 << 30)) return ATTN_ERR_INVALID;
+    if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o_part, 16) ||
+        !aligned(lse_part, 4))
+        return ATTN_ERR_ALIGN;
+    const int diag = causal ? diag_offset : s_k - s_q;
+    // Causal rows 0 .. -diag - 1 see no key of the shard: their partial is
+    // written by a fill launch first (the forward skips wholly empty blocks).
+    const long long n_empty = causal ? (diag < 0 ? (-static_cast<long long>(diag) < s_q
+                                                         ? -static_cast<long long>(diag)
+                                                         : s_q)
+                                                  : 0)
+                                     : 0;
+    int launches = 0;
+    if (n_empty > 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+        DeviceState* st = nullptr;
+        rc = init_device(dev, &st);
+        if (rc != ATTN_OK) return rc;
+        const size_t rows = static_cast<size_t>(batch) * h_q * n_empty;
+        size_t blocks = (rows + kMergeThreads / 32 - 1) / (kMergeThreads / 32);
+        const size_t cap = static_cast<size_t>(st->num_sms) * 8;
+        if (blocks > cap) blocks = cap;
+        attn_fill_empty_rows_kernel<<<static_cast<unsigned>(blocks), kMergeThreads, 0,
+                                      static_cast<cudaStream_t>(stream)>>>(
+            o_part, lse_part, batch, h_q, s_q, static_cast<int>(n_empty));
+        if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+        ++launches;
+    }
+    if (n_empty < s_q) {
+        const int n_kb = (s_k + kBlockN - 1) / kBlockN;
+        rc = launch_fwd(q, k, v, nullptr, nullptr, batch, h_q, h_kv, s_q, s_k, causal, diag,
+                        scale, 1, n_kb, o_part, lse_part, stream);
+        if (rc != ATTN_OK) return rc;
+        ++launches;
+    }
+    g_last_launches = launches;
+    return ATTN_OK;
 }
 
 extern "C" int attn_merge_partials(const float* o_parts, const float* lse_parts, int n_parts,

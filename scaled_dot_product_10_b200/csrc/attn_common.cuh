@@ -50,7 +50,8 @@ struct FwdParams {
     int n_kb;     // ceil(s_k / 128)
     int n_pairs;  // ceil(n_qb / 2): CTA tiles per (batch, head)
     int causal;
-    int causal_offset;      // s_k - s_q: causal row i sees keys 0 .. i + causal_offset
+    int causal_offset;      // causal row i sees keys 0 .. i + causal_offset: s_k - s_q,
+                            // or a key shard's diagonal (may be negative)
     int num_tiles;          // work items: pairs x n_splits
     int units_per_section;  // (batch, kv head) units whose K/V share L2 at once
     int n_splits;           // key ranges per pair (1: the whole key sequence)
@@ -83,6 +84,7 @@ struct FwdParams {
     float* lse_part;
     unsigned long long timeout_ns;
     unsigned int* status;
+    int window_left;  // sliding window (windowed kernel only): keys before the diagonal
 };
 
 // ------------------------------------------------------------------ waits

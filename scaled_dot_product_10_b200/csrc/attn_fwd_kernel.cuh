@@ -71,6 +71,12 @@ constexpr uint32_t kRegsSoftmax = 216;
 constexpr uint32_t kRegsControl = 72;
 
 // ------------------------------------------------------------------ schedule
+// Items are dealt to the G = gridDim.x persistent CTAs in rounds of G, in a
+// snake order: in round k CTA c takes item kG + c when k is even and
+// kG + G - 1 - c when k is odd.  Items run longest first (below), so a CTA
+// that took a long item in one round takes a short one in the next and the
+// causal work per CTA evens out (a plain grid stride gives CTA 0 the longest
+// item of every round).
 // Work item t -> (pair, key range): pair u = t / n_splits, key range
 // t % n_splits (the ranges of one pair are adjacent, so they share its Q
 // tiles in L2).  Pair u -> (batch, query head, first query block): pairs are
@@ -80,11 +86,19 @@ constexpr uint32_t kRegsControl = 72;
 // the query heads of the unit's group (adjacent heads share K/V).  Items
 // whose key range no row of the pair may see (causal) are skipped by every
 // role alike.
+//
+// With a sliding window (kWindow) the two query blocks of a pair see
+// different key intervals: iteration t of the pair's K/V stream is key block
+// kb0 + t; block 0 visits iterations 0 .. n[0] - 1 and block 1 iterations
+// st1 .. st1 + n[1] - 1 (its window starts st1 key blocks later).
+template <bool kWindow>
 struct PairCursor {
+    int round;  // rounds of gridDim.x items dealt so far
     int t;
     int b, h, g, qb0;
     int split, kb0;  // key range of the item: key blocks kb0 .. kb0 + n[i] - 1
     int n[2];        // key/value blocks each query block of the pair visits (0: none)
+    int st1;         // kWindow: first iteration of block 1 (0 otherwise)
 
     __device__ __forceinline__ void decode(const FwdParams& p) {
         const int u = p.div_splits.div(t);
@@ -106,32 +120,60 @@ struct PairCursor {
         g = unit - b * p.h_kv;
         h = g * p.group + h_local;
         qb0 = 2 * pair;
-        // Causal (bottom-right aligned, s_q <= s_k): the last row of block
-        // qb, min(128 qb + 127, s_q - 1), sees keys up to row + s_k - s_q.
-        const int last0 = (min(qb0 * kBlockM + kBlockM - 1, p.s_q - 1) + p.causal_offset) / kBlockN;
-        const int last1 = (min(qb0 * kBlockM + 2 * kBlockM - 1, p.s_q - 1) + p.causal_offset) / kBlockN;
+        // Causal: the last row of block qb, min(128 qb + 127, s_q - 1), sees
+        // keys up to row + causal_offset (s_k - s_q, or a key shard's own
+        // diagonal, which may be negative: floor division by the shift).
+        static_assert(kBlockN == 128, "the shift below divides by kBlockN");
+        const int last0 = (min(qb0 * kBlockM + kBlockM - 1, p.s_q - 1) + p.causal_offset) >> 7;
+        const int last1 = (min(qb0 * kBlockM + 2 * kBlockM - 1, p.s_q - 1) + p.causal_offset) >> 7;
         const int vis0 = p.causal ? min(kb_end, last0 + 1) : kb_end;
         const int vis1 = (qb0 + 1 < p.n_qb) ? (p.causal ? min(kb_end, last1 + 1) : kb_end) : 0;
         n[0] = max(0, vis0 - kb0);
         n[1] = max(0, vis1 - kb0);
+        if constexpr (kWindow) {
+            // Causal with a window of window_left keys before the diagonal
+            // (no key ranges): row r sees keys r + causal_offset -
+            // window_left .. r + causal_offset, so a block starts at the key
+            // block of its first row's lower bound.
+            const int lo0 = max(0, (qb0 * kBlockM + p.causal_offset - p.window_left) >> 7);
+            const int lo1 = max(0, ((qb0 + 1) * kBlockM + p.causal_offset - p.window_left) >> 7);
+            kb0 = lo0;
+            n[0] = vis0 - lo0;
+            st1 = lo1 - lo0;
+            n[1] = (qb0 + 1 < p.n_qb) ? vis1 - lo1 : 0;
+        } else {
+            st1 = 0;
+        }
     }
-    // Decode item t, moving on (by the grid stride) past items with no work.
+    // This CTA's item of the current round, moving on past items with no
+    // work.  Positions only grow from round to round, so the first one past
+    // the last item ends the walk.
     __device__ __forceinline__ void settle(const FwdParams& p) {
-        for (; t < p.num_tiles; t += gridDim.x) {
+        for (;; ++round) {
+            const int c = static_cast<int>(blockIdx.x);
+            const int g = static_cast<int>(gridDim.x);
+            t = round * g + ((round & 1) ? g - 1 - c : c);
+            if (t >= p.num_tiles) return;
             decode(p);
             if (n[0] > 0 || n[1] > 0) return;
         }
     }
     __device__ __forceinline__ void start(const FwdParams& p) {
-        t = blockIdx.x;
+        round = 0;
         settle(p);
     }
     __device__ __forceinline__ void next(const FwdParams& p) {
-        t += gridDim.x;
+        ++round;
         settle(p);
     }
     __device__ __forceinline__ bool valid(const FwdParams& p) const { return t < p.num_tiles; }
-    __device__ __forceinline__ int iters() const { return max(n[0], n[1]); }
+    __device__ __forceinline__ int iters() const {
+        if constexpr (kWindow) return max(n[0], st1 + n[1]);
+        return max(n[0], n[1]);
+    }
+    // Iterations both blocks visit, [common_begin, common_end) (may be empty).
+    __device__ __forceinline__ int common_begin() const { return st1; }
+    __device__ __forceinline__ int common_end() const { return min(n[0], st1 + n[1]); }
 };
 
 // ------------------------------------------------------------------ layout
@@ -197,6 +239,7 @@ __device__ __forceinline__ void exp_row(const float (&s)[128], uint64_t c2x2, ui
 
 // ------------------------------------------------------------------ softmax
 // One softmax warpgroup: thread r owns query row r of its block (TMEM lane r).
+template <bool kWindow>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorMap* tm_o,
                                              const WaitCtx& wc, uint32_t tmem, uint32_t sP,
                                              uint32_t bars, int wg, int warp_in_wg, int lane) {
@@ -227,11 +270,20 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
     uint32_t cnt = 0;     // S blocks this warpgroup has processed (all pairs)
     uint32_t stored = 0;  // O tiles this warpgroup has stored through TMA
     uint32_t rounds = 0;  // alternation rounds before this pair
-    PairCursor c;
+    PairCursor<kWindow> c;
     c.start(p);
     for (; c.valid(p); c.next(p)) {
         const int n = c.n[wg];
-        const int n_turns = min(c.n[0], c.n[1]);
+        int n_turns, t0 = 0, cb = 0;
+        if constexpr (kWindow) {
+            // Turns over the iterations both blocks visit; this block's
+            // local step j is iteration t0 + j.
+            cb = c.common_begin();
+            n_turns = max(0, c.common_end() - cb);
+            t0 = wg ? c.st1 : 0;
+        } else {
+            n_turns = min(c.n[0], c.n[1]);
+        }
         const uint32_t round0 = rounds;
         rounds += static_cast<uint32_t>(n_turns);
         if (n == 0) continue;
@@ -256,17 +308,30 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(b_sfree);
 
-            const int kv0 = (c.kb0 + j) * kBlockN;
+            const int kv0 = (c.kb0 + t0 + j) * kBlockN;
             const bool diag = p.causal && (kv0 + kBlockN - 1 > qb * kBlockM + p.causal_offset);
-            const bool masked = diag || kv0 + kBlockN > p.s_k;
+            bool masked = diag || kv0 + kBlockN > p.s_k;
+            if constexpr (kWindow) {
+                // keys before the last row's window start
+                masked = masked ||
+                         kv0 < qb * kBlockM + kBlockM - 1 + p.causal_offset - p.window_left;
+            }
             if (masked) {
                 const int lim_tail = p.s_k - kv0;                           // keys >= s_k
                 // keys past row + s_k - s_q
                 const int lim_causal = p.causal ? row + p.causal_offset - kv0 + 1 : kBlockN;
                 const int lim = min(lim_tail, lim_causal);
+                if constexpr (kWindow) {
+                    // and keys before row + s_k - s_q - window_left
+                    const int lo = row + p.causal_offset - p.window_left - kv0;
 #pragma unroll
-                for (int k = 0; k < 128; ++k)
-                    if (k >= lim) s[k] = -CUDART_INF_F;
+                    for (int k = 0; k < 128; ++k)
+                        if (k >= lim || k < lo) s[k] = -CUDART_INF_F;
+                } else {
+#pragma unroll
+                    for (int k = 0; k < 128; ++k)
+                        if (k >= lim) s[k] = -CUDART_INF_F;
+                }
             }
             float mx;
             {
@@ -323,8 +388,16 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
             }
 
             // Our turn on the exponential unit: wait for turn m - 1.
-            const bool turn = j < n_turns;
-            const uint32_t m = 2 * (round0 + j) + wg;
+            bool turn;
+            uint32_t m;
+            if constexpr (kWindow) {
+                const int tc = t0 + j - cb;  // position in the common interval
+                turn = tc >= 0 && tc < n_turns;
+                m = 2 * (round0 + tc) + wg;
+            } else {
+                turn = j < n_turns;
+                m = 2 * (round0 + j) + wg;
+            }
             if (turn && m > 0 && !wait_bar_warp(b_turn, (m - 1) & 1, wc)) return;
             float sum_a = 0.f, sum_b = 0.f;
             exp_row(s, c2x2, ptx::f2_pack(neg_mc, neg_mc), p_row, p_xor, sum_a, sum_b, turn, b_turn,
@@ -345,6 +418,10 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
                 const float lse_row = (m_ref * c2 + __log2f(l_run)) * 0.69314718055994531f;
                 const size_t row_id = (static_cast<size_t>(c.b) * p.h_q + c.h) * p.s_q + row;
                 if (p.o_part != nullptr) {
+                    // A row of a key shard may see none of its keys (l = 0):
+                    // O = 0 and LSE = -inf, so a merge gives it no weight.
+                    const float inv_lp = l_run > 0.f ? inv_l : 0.f;
+                    const uint64_t il2p = ptx::f2_pack(inv_lp, inv_lp);
                     const size_t part =
                         static_cast<size_t>(c.split) * p.batch * p.h_q * p.s_q + row_id;
                     float4* frow = reinterpret_cast<float4*>(p.o_part + part * kHeadDim);
@@ -359,11 +436,11 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
                                 float a0, a1, b0, b1;
                                 ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(__uint_as_float(ov[4 * k]),
                                                                         __uint_as_float(ov[4 * k + 1])),
-                                                           il2),
+                                                           il2p),
                                                a0, a1);
                                 ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(__uint_as_float(ov[4 * k + 2]),
                                                                         __uint_as_float(ov[4 * k + 3])),
-                                                           il2),
+                                                           il2p),
                                                b0, b1);
                                 frow[q * 8 + k] = make_float4(a0, a1, b0, b1);
                             }
@@ -429,6 +506,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
 }
 
 // ------------------------------------------------------------------ kernel
+template <bool kWindow>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -503,14 +581,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t k_loads = 0, v_loads = 0;  // K / V tiles issued
             uint32_t q_loads[2] = {0, 0};
             bool ok = true;
-            auto load_tile = [&](const CUtensorMap* tm, uint32_t dst, uint32_t full, const PairCursor& c,
+            auto load_tile = [&](const CUtensorMap* tm, uint32_t dst, uint32_t full,
+                                 const PairCursor<kWindow>& c,
                                  int j) {
                 ptx::mbar_arrive_expect_tx(full, kTileBytes);
                 const int key0 = (c.kb0 + j) * kBlockN;
                 ptx::tma_load_4d(dst, tm, full, 0, c.g, key0, c.b, pol_kv);
                 ptx::tma_load_4d(dst + kHalfTileBytes, tm, full, 64, c.g, key0, c.b, pol_kv);
             };
-            auto load_k = [&](const PairCursor& c, int j) -> bool {
+            auto load_k = [&](const PairCursor<kWindow>& c, int j) -> bool {
                 const int slot = k_loads % kKStages;
                 if (!wait_bar(bar(L::bKEmpty + slot), ((k_loads / kKStages) & 1) ^ 1, wc))
                     return false;
@@ -518,7 +597,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++k_loads;
                 return true;
             };
-            auto load_v = [&](const PairCursor& c, int j) -> bool {
+            auto load_v = [&](const PairCursor<kWindow>& c, int j) -> bool {
                 const int slot = v_loads % kVStages;
                 if (!wait_bar(bar(L::bVEmpty + slot), ((v_loads / kVStages) & 1) ^ 1, wc))
                     return false;
@@ -526,7 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++v_loads;
                 return true;
             };
-            PairCursor c;
+            PairCursor<kWindow> c;
             c.start(p);
             for (; ok && c.valid(p); c.next(p)) {
 #pragma unroll
@@ -648,11 +727,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++pv_cnt;
                 return true;
             };
-            PairCursor c;
+            PairCursor<kWindow> c;
             c.start(p);
             for (; ok && c.valid(p); c.next(p)) {
                 const int n = c.iters();
                 const int ni = c.n[i];
+                if constexpr (kWindow) {
+                    // Block i visits iterations [st, st + ni) of the pair's
+                    // K/V stream; other tiles are passed on.  Tile order (the
+                    // producer's): K(0), then per step j: K(j+1), V(j).
+                    const int st = i ? c.st1 : 0;
+                    auto in_range = [&](int t) { return ni > 0 && t >= st && t < st + ni; };
+                    auto scores = [&](int t) -> bool {
+                        if (!in_range(t)) return skip_k();
+                        if (t == st) {
+                            if (!wait_bar(bar(L::bQFull + i), started & 1, wc)) return false;
+                            ++started;
+                        }
+                        return qk(t == st + ni - 1);
+                    };
+                    if (!(ok = scores(0))) break;
+                    for (int j = 0; j < n && ok; ++j) {
+                        if (j + 1 < n && !(ok = scores(j + 1))) break;
+                        if (in_range(j)) {
+                            if (j == st && started > 1 &&
+                                !(ok = wait_bar(bar(L::bOEmpty + i), started & 1, wc)))
+                                break;
+                            ok = pv(j > st);
+                        } else {
+                            ok = skip_v();
+                        }
+                    }
+                    continue;
+                }
                 // Tile order (the producer's): K0, then per step j: K(j+1), V(j).
                 if (ni > 0) {
                     if (!(ok = wait_bar(bar(L::bQFull + i), started & 1, wc))) break;
@@ -683,7 +790,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp < 8) {
         ptx::reg_alloc<kRegsSoftmax>();
-        softmax_role(p, &tm_o, wc, tmem, sP, bars, warp >> 2, warp & 3, lane);
+        softmax_role<kWindow>(p, &tm_o, wc, tmem, sP, bars, warp >> 2, warp & 3, lane);
     } else {
         ptx::reg_dealloc<kRegsControl>();  // idle warps of the control warpgroup
     }

@@ -81,3 +81,26 @@ __global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const MergePa
 }
 
 }  // namespace sdpa10
+
+namespace sdpa10 {
+
+// Partials of a key shard under the causal mask: query rows 0 .. n_empty - 1
+// see none of the shard's keys.  The forward skips their blocks when whole
+// blocks are empty, so this writes their partial (O = 0, LSE = -inf: no
+// weight in a merge).  One warp per row, 16 bytes per lane; memory-bound.
+__global__ void __launch_bounds__(kMergeThreads)
+    attn_fill_empty_rows_kernel(float* o_part, float* lse_part, int batch, int h_q, int s_q,
+                                int n_empty) {
+    const int lane = threadIdx.x & 31;
+    const size_t rows = static_cast<size_t>(batch) * h_q * n_empty;
+    const size_t warps = static_cast<size_t>(gridDim.x) * (kMergeThreads / 32);
+    for (size_t r = blockIdx.x * static_cast<size_t>(kMergeThreads / 32) + (threadIdx.x >> 5);
+         r < rows; r += warps) {
+        const size_t bh = r / n_empty;
+        const size_t row = bh * s_q + (r - bh * n_empty);  // [batch][h_q][s_q] row index
+        reinterpret_cast<float4*>(o_part + row * 128)[lane] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane == 0) lse_part[row] = -CUDART_INF_F;
+    }
+}
+
+}  // namespace sdpa10

@@ -202,3 +202,14 @@ def test_python_binding_requires_cuda_tensors():
 def test_missing_library_fails_loudly(tmp_path):
     with pytest.raises(OSError):
         attn.load_library(str(tmp_path / "nope.so"))
+
+
+def test_window_entry_validation(lib):
+    f = lib.attn_fwd_window
+    ok = (A, A, A, A, A, 1, 2, 2, 256, 256, 128)
+    assert f(*ok, -1, 0.088, None) == attn.ATTN_ERR_INVALID
+    assert f(*ok[:10], 64, 10, 0.088, None) == attn.ATTN_ERR_UNSUPPORTED
+    assert f(A, A, A, A, A, 1, 2, 2, 512, 256, 128, 10, 0.088, None) == attn.ATTN_ERR_UNSUPPORTED
+    assert f(A + 8, *ok[1:], 10, 0.088, None) == attn.ATTN_ERR_ALIGN
+    if not torch.cuda.is_available():
+        assert f(*ok, 10, 0.088, None) == attn.ATTN_ERR_CUDA

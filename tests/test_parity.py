@@ -228,3 +228,61 @@ def test_workload_configs(name, causal):
     rows = _rows_for(w, 512) if w.sampled else None
     m = check(q, k, v, causal, w.scale, rows=rows, what=f"{name} causal={causal}")
     print(name, causal, m)
+
+
+# ------------------------------------------------------------ sliding window
+def check_window(q, k, v, w, scale=SCALE, rows=None, what=""):
+    o, lse = attn.attn_fwd_window(q.cuda(), k.cuda(), v.cuda(), w, scale=scale)
+    rc = attn.attn_status()
+    assert rc == attn.ATTN_OK, attn.attn_strerror(rc)
+    o_ref, l_ref, _ = oracle.attn_fwd(q, k, v, True, scale, rows=rows, window_left=w)
+    oo, ll = gather_rows(o, lse, rows)
+    m = metrics(oo, ll, o_ref, l_ref)
+    assert_within(m, what)
+    return o, lse
+
+
+@pytest.mark.parametrize("s_q,s_k,w", [
+    (1000, 1000, 0), (1000, 1000, 1), (1000, 1000, 127), (1000, 1000, 128),
+    (1000, 1000, 129), (1000, 1000, 300), (640, 640, 255), (129, 129, 64),
+    (300, 1000, 100),   # bottom-right: the window slides with the offset
+    (1, 4096, 500),     # one query row
+    (2048, 2048, 2047), # the window covers every visible key
+])
+def test_window_matches_oracle(s_q, s_k, w):
+    q, k, v = make_qkv(2, 4, 2, s_q, s_k, seed=9000 + s_q + w)
+    check_window(q, k, v, w, what=f"window {s_q}x{s_k} w={w}")
+
+
+@pytest.mark.parametrize("h_q,h_kv", [(16, 2), (16, 1)])
+def test_window_head_sharing(h_q, h_kv):
+    q, k, v = make_qkv(2, h_q, h_kv, 2048, 2048, seed=9100 + h_kv)
+    rows = sample_rows(2, h_q, 2048, 128, seed=9101)
+    check_window(q, k, v, 511, rows=rows, what=f"window gqa {h_q}/{h_kv}")
+
+
+def test_window_wider_than_keys_is_causal_bit_exact():
+    q, k, v = make_qkv(1, 4, 4, 700, 700, seed=9200)
+    o1, l1 = run_gpu(q, k, v, True, SCALE)
+    o2, l2 = attn.attn_fwd_window(q.cuda(), k.cuda(), v.cuda(), 5000, scale=SCALE)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+
+
+@pytest.mark.parametrize("s,w", [(4096, 1000), (3968, 300), (1152, 129)])
+def test_window_turn_order_many_launches(s, w):
+    # Windowed pairs take turns only over the key blocks both query blocks
+    # visit; 100 launches must give a clean status word and identical bits.
+    b, h = 2, 16
+    q, k, v = make_qkv(b, h, h, s, s, seed=9300 + s)
+    qd, kd, vd = q.cuda(), k.cuda(), v.cuda()
+    o0, l0 = attn.attn_fwd_window(qd, kd, vd, w, scale=SCALE)
+    o, lse = torch.empty_like(o0), torch.empty_like(l0)
+    for i in range(100):
+        attn.attn_fwd_window(qd, kd, vd, w, scale=SCALE, o=o, lse=lse)
+        if i % 50 == 49:
+            assert attn.attn_status() == attn.ATTN_OK, f"launch {i}"
+            assert torch.equal(o, o0) and torch.equal(lse, l0), f"launch {i}"
+    rows = sample_rows(b, h, s, 64, seed=9310 + s)
+    o_ref, l_ref, _ = oracle.attn_fwd(q, k, v, True, SCALE, rows=rows, window_left=w)
+    oo, ll = gather_rows(o0, l0, rows)
+    assert_within(metrics(oo, ll, o_ref, l_ref), f"window s={s} w={w}")

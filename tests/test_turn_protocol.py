@@ -38,6 +38,37 @@ def ops_strict(pairs, wg):
     return ops
 
 
+def ops_window(pairs, wg):
+    """The kernel's rule for windowed pairs (n0, st1, n1): block 1 visits
+    iterations st1 .. st1 + n1 - 1 of the pair's stream, block 0 iterations
+    0 .. n0 - 1; turns alternate over the iterations both visit."""
+    ops, rounds = [], 0
+    for n0, st1, n1 in pairs:
+        cb, ce = st1, min(n0, st1 + n1)
+        n_turns = max(0, ce - cb)
+        t0, n = (0, n0) if wg == 0 else (st1, n1)
+        for j in range(n):
+            tc = t0 + j - cb
+            if 0 <= tc < n_turns:
+                m = 2 * (rounds + tc) + wg
+                ops.append((m - 1 if m > 0 else None, m))
+        rounds += n_turns
+    return ops
+
+
+def random_window_pairs(rng, n_pairs):
+    """(n0, st1, n1) as the windowed cursor produces them: block 1's window
+    starts st1 >= 0 key blocks later and ends at or after block 0's."""
+    pairs = []
+    for _ in range(n_pairs):
+        n0 = rng.randint(1, 6)
+        st1 = rng.randint(0, n0 + 1)
+        end1 = max(n0, st1 + 1) + rng.randint(0, 1)
+        n1 = 0 if rng.randrange(6) == 0 else end1 - st1
+        pairs.append((n0, st1, n1))
+    return pairs
+
+
 def ops_global_sequence(pairs, wg):
     """The planted mistake: every exponential phase of either block takes the
     next number of one global sequence (block 0 first at each key step)."""
@@ -144,3 +175,21 @@ def test_global_sequence_rule_fails_on_causal_pairs(pairs):
     o0, o1 = ops_global_sequence(pairs, 0), ops_global_sequence(pairs, 1)
     results = {simulate(o0, o1, rng) for _ in range(200)}
     assert "early" in results or "stuck" in results
+
+
+def test_window_turn_rule_is_safe_under_every_interleaving():
+    rng = random.Random(7)
+    for _ in range(400):
+        pairs = random_window_pairs(rng, rng.randint(1, 8))
+        o0, o1 = ops_window(pairs, 0), ops_window(pairs, 1)
+        for _ in range(20):
+            assert simulate(o0, o1, rng) == "ok", pairs
+
+
+def test_window_rule_reduces_to_the_unwindowed_rule():
+    rng = random.Random(8)
+    for _ in range(200):
+        pairs = random_pairs(rng, rng.randint(1, 8))
+        pairs = [(n0, 0, n1) for n0, n1 in pairs if n0 > 0]
+        for wg in (0, 1):
+            assert ops_window(pairs, wg) == ops_strict([(a, c) for a, _, c in pairs], wg)
