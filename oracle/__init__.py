@@ -51,6 +51,13 @@ def load(path: str | None = None):
         ctypes.c_void_p, ctypes.c_int,
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
     ]
+    lib.oracle_attn_bwd_f64.restype = ctypes.c_int
+    lib.oracle_attn_bwd_f64.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_double,
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+    ]
     lib.oracle_num_threads.restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -155,3 +162,26 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, causal: bool, scale: fl
         o[q0:q1] = ob[0].transpose(1, 0, 2)
         lse[:, q0:q1] = lb[0]
     return o, lse
+
+
+def attn_bwd(q, k, v, dout, causal: bool, scale: float, window_left: int = -1, lib=None):
+    """Gradients of the forward: given dO (the gradient of a loss with
+    respect to O), returns (dq, dk, dv) as float64 arrays in the layouts of
+    q, k and v ([batch, s, heads, d]).  q, k, v, dout: bf16 (torch tensors
+    or uint16 bits), dout shaped like q."""
+    qb, kb, vb, ob = _as_bits(q), _as_bits(k), _as_bits(v), _as_bits(dout)
+    batch, s_q, h_q, d = qb.shape
+    bk, s_k, h_kv, dk_ = kb.shape
+    if vb.shape != kb.shape or bk != batch or dk_ != d or ob.shape != qb.shape:
+        raise ValueError("shape mismatch between q, k, v and dout")
+    dq = np.zeros((batch, s_q, h_q, d), dtype=np.float64)
+    dk = np.zeros((batch, s_k, h_kv, d), dtype=np.float64)
+    dv = np.zeros((batch, s_k, h_kv, d), dtype=np.float64)
+    lib = lib or load()
+    rc = lib.oracle_attn_bwd_f64(qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, ob.ctypes.data,
+                                 batch, h_q, h_kv, s_q, s_k, d, int(bool(causal)),
+                                 int(window_left), float(scale), dq.ctypes.data, dk.ctypes.data,
+                                 dv.ctypes.data)
+    if rc != 0:
+        raise ValueError(f"oracle rejected its arguments (code {rc})")
+    return dq, dk, dv

@@ -199,3 +199,148 @@ int oracle_num_threads(void)
     return 1;
 #endif
 }
+
+/*
+ * ---------------------------------------------------------------------------
+ * Backward pass (gradients of the forward above).  TEST INFRASTRUCTURE ONLY,
+ * like the forward.
+ *
+ * The pages describe FlashAttention's backward as recomputing the attention
+ * weights from saved row statistics instead of storing them (bjdmk.com.cn
+ * survey page, section 5.1) and reusing the forward's intermediates
+ * (intelliparadigm.com AVO page, section 3.2).  What the backward computes is
+ * fixed by the chain rule applied to the forward's definition; this is that
+ * definition written out, with P materialised from scratch (no saved
+ * statistics are taken from the caller):
+ *
+ *   P   = softmax_rows(scale * Q K^T + mask)      (as in the forward)
+ *   dV  = P^T dO                                   dV[j] = sum_i P[i][j] dO[i]
+ *   dP  = dO V^T                                   dP[i][j] = dO[i] . V[j]
+ *   D_i = sum_j P[i][j] dP[i][j]
+ *   dS  = P * (dP - D)                             (elementwise, D per row)
+ *   dQ  = scale * dS K                             dQ[i] = scale sum_j dS[i][j] K[j]
+ *   dK  = scale * dS^T Q                           dK[j] = scale sum_i dS[i][j] Q[i]
+ *
+ * (the softmax Jacobian dS[i][j] = sum_k dP[i][k] P[i][k] (delta_jk - P[i][j])
+ * gives the dS line).  Grouped heads: dK and dV of key/value head g sum the
+ * contributions of every query head h with h / (h_q / h_kv) = g.
+ *
+ * Layouts: q, do bf16 bits [batch][s_q][h_q][d]; k, v [batch][s_k][h_kv][d];
+ * dq double [batch][s_q][h_q][d]; dk, dv double [batch][s_k][h_kv][d].
+ * causal / window_left as the forward.  Returns 0, or a negative code on a
+ * bad argument (-7: out of memory).
+ */
+static void backward_group(const double *Q, const double *K, const double *V, const double *dO,
+                           int b, int g, int h_q, int h_kv, int s_q, int s_k, int d,
+                           int causal, int window_left, double scale,
+                           double *dq, double *dk, double *dv, double *P, double *dP)
+{
+    const int group = h_q / h_kv;
+    const int64_t qs = (int64_t)h_q * d, ks = (int64_t)h_kv * d;
+    const int off = s_k - s_q;
+    const double *Kb = K + (int64_t)b * s_k * ks + (int64_t)g * d;
+    const double *Vb = V + (int64_t)b * s_k * ks + (int64_t)g * d;
+    double *dKb = dk + (int64_t)b * s_k * ks + (int64_t)g * d;
+    double *dVb = dv + (int64_t)b * s_k * ks + (int64_t)g * d;
+
+    for (int h = g * group; h < (g + 1) * group; ++h) {
+        const double *Qb = Q + (int64_t)b * s_q * qs + (int64_t)h * d;
+        const double *dOb = dO + (int64_t)b * s_q * qs + (int64_t)h * d;
+        double *dQb = dq + (int64_t)b * s_q * qs + (int64_t)h * d;
+
+        /* P, row by row (the forward's steps 1 and 2) */
+        for (int i = 0; i < s_q; ++i) {
+            double *Prow = P + (int64_t)i * s_k;
+            for (int j = 0; j < s_k; ++j) {
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += Qb[(int64_t)i * qs + c] * Kb[(int64_t)j * ks + c];
+                Prow[j] = scale * dot;
+                if (causal && j > i + off) Prow[j] = -INFINITY;
+                if (window_left >= 0 && j < i + off - window_left) Prow[j] = -INFINITY;
+            }
+            double m = -INFINITY;
+            for (int j = 0; j < s_k; ++j)
+                if (Prow[j] > m) m = Prow[j];
+            double l = 0.0;
+            for (int j = 0; j < s_k; ++j) {
+                Prow[j] = exp(Prow[j] - m);
+                l += Prow[j];
+            }
+            for (int j = 0; j < s_k; ++j) Prow[j] = Prow[j] / l;
+        }
+        /* dP = dO V^T, D_i = sum_j P dP, dS = P (dP - D) (stored over dP) */
+        for (int i = 0; i < s_q; ++i) {
+            const double *Prow = P + (int64_t)i * s_k;
+            double *dProw = dP + (int64_t)i * s_k;
+            for (int j = 0; j < s_k; ++j) {
+                double dot = 0.0;
+                for (int c = 0; c < d; ++c) dot += dOb[(int64_t)i * qs + c] * Vb[(int64_t)j * ks + c];
+                dProw[j] = dot;
+            }
+            double Di = 0.0;
+            for (int j = 0; j < s_k; ++j) Di += Prow[j] * dProw[j];
+            for (int j = 0; j < s_k; ++j) dProw[j] = Prow[j] * (dProw[j] - Di);
+        }
+        /* dQ = scale dS K */
+        for (int i = 0; i < s_q; ++i) {
+            const double *dSrow = dP + (int64_t)i * s_k;
+            for (int c = 0; c < d; ++c) {
+                double acc = 0.0;
+                for (int j = 0; j < s_k; ++j) acc += dSrow[j] * Kb[(int64_t)j * ks + c];
+                dQb[(int64_t)i * qs + c] = scale * acc;
+            }
+        }
+        /* dK += scale dS^T Q;  dV += P^T dO  (summed over the group's heads) */
+        for (int j = 0; j < s_k; ++j) {
+            for (int c = 0; c < d; ++c) {
+                double acc_k = 0.0, acc_v = 0.0;
+                for (int i = 0; i < s_q; ++i) {
+                    acc_k += dP[(int64_t)i * s_k + j] * Qb[(int64_t)i * qs + c];
+                    acc_v += P[(int64_t)i * s_k + j] * dOb[(int64_t)i * qs + c];
+                }
+                dKb[(int64_t)j * ks + c] += scale * acc_k;
+                dVb[(int64_t)j * ks + c] += acc_v;
+            }
+        }
+    }
+}
+
+int oracle_attn_bwd_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
+                        const uint16_t *dout, int batch, int h_q, int h_kv, int s_q, int s_k,
+                        int d, int causal, int window_left, double scale,
+                        double *dq, double *dk, double *dv)
+{
+    if (!q || !k || !v || !dout || !dq || !dk || !dv) return -1;
+    if (batch <= 0 || h_q <= 0 || h_kv <= 0 || s_q <= 0 || s_k <= 0 || d <= 0) return -2;
+    if (h_q % h_kv != 0) return -3;
+    if (causal && s_q > s_k) return -6;
+    if (window_left < -1 || (window_left >= 0 && !causal)) return -8;
+
+    const int64_t nq = (int64_t)batch * s_q * h_q * d, nk = (int64_t)batch * s_k * h_kv * d;
+    double *Q = decode_bf16(q, nq), *K = decode_bf16(k, nk), *V = decode_bf16(v, nk);
+    double *dO = decode_bf16(dout, nq);
+    if (!Q || !K || !V || !dO) { free(Q); free(K); free(V); free(dO); return -7; }
+    for (int64_t t = 0; t < nk; ++t) { dk[t] = 0.0; dv[t] = 0.0; }
+
+    const int64_t n_tasks = (int64_t)batch * h_kv;
+    int failed = 0;
+#pragma omp parallel
+    {
+        double *P = (double *)malloc((size_t)s_q * s_k * sizeof(double));
+        double *dP = (double *)malloc((size_t)s_q * s_k * sizeof(double));
+        if (!P || !dP) {
+#pragma omp atomic write
+            failed = 1;
+        }
+#pragma omp for schedule(dynamic, 1)
+        for (int64_t t = 0; t < n_tasks; ++t) {
+            if (!P || !dP) continue;
+            backward_group(Q, K, V, dO, (int)(t / h_kv), (int)(t % h_kv), h_q, h_kv, s_q, s_k, d,
+                           causal, window_left, scale, dq, dk, dv, P, dP);
+        }
+        free(P);
+        free(dP);
+    }
+    free(Q); free(K); free(V); free(dO);
+    return failed ? -7 : 0;
+}

@@ -372,6 +372,96 @@ def pin_varlen_sequences_are_independent(lib):
     assert np.all(np.abs(o2[cu_q[1]:cu_q[2]] + 0.5) < 1e-14)
 
 
+# ------------------------------------------------------------------ backward
+def _torch_grads(q, k, v, dout, scale, mask=None):
+    """dQ, dK, dV from torch's float64 autograd of its SDPA (an independent
+    library routine), for L = sum(O * dO); layouts as the oracle's."""
+    qt = q.double().permute(0, 2, 1, 3).requires_grad_()
+    kt = k.double().permute(0, 2, 1, 3).requires_grad_()
+    vt = v.double().permute(0, 2, 1, 3).requires_grad_()
+    o = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=scale,
+                                                         enable_gqa=True)
+    (o * dout.double().permute(0, 2, 1, 3)).sum().backward()
+    return tuple(t.grad.permute(0, 2, 1, 3).numpy() for t in (qt, kt, vt))
+
+
+def pin_bwd_torch_autograd_f64(lib):
+    """Backward = torch float64 autograd of SDPA: MHA and GQA, non-causal,
+    bottom-right causal and a sliding window (as explicit boolean masks)."""
+    for (hq, hkv, sq, sk, causal, w, seed) in [(4, 4, 21, 21, False, -1, 41),
+                                              (4, 2, 19, 30, True, -1, 42),
+                                              (6, 3, 25, 25, True, 5, 43),
+                                              (2, 1, 1, 17, True, -1, 44)]:
+        q, k, v = make_qkv(2, hq, hkv, sq, sk, seed=seed, d=16)
+        dout = make_qkv(2, hq, hkv, sq, sk, seed=seed + 100, d=16)[0]
+        mask = None
+        if causal:
+            i = torch.arange(sq)[:, None]
+            j = torch.arange(sk)[None, :]
+            mask = j <= i + (sk - sq)
+            if w >= 0:
+                mask &= j >= i + (sk - sq) - w
+        got = oracle.attn_bwd(q, k, v, dout, causal, 0.35, window_left=w, lib=lib)
+        want = _torch_grads(q, k, v, dout, 0.35, mask)
+        for name, g, t in zip(("dQ", "dK", "dV"), got, want):
+            assert np.max(np.abs(g - t)) < 1e-11, f"{name} vs torch autograd ({hq}/{hkv})"
+
+
+def pin_bwd_finite_differences(lib):
+    """Central differences of the (pinned) forward oracle: for
+    L = sum(O * dO), dL/dx ~ (L(x + e) - L(x - e)) / 2e.  Inputs and steps sit
+    on a 2^-6 grid, so x +- e stays exact in BF16."""
+    rng = np.random.default_rng(45)
+    b, hq, hkv, sq, sk, d, scale = 1, 2, 1, 9, 11, 8, 0.4
+    e = 2.0 ** -6
+    base = [grid_values(rng, shp, -1.0, 1.0, e) for shp in
+            ((b, sq, hq, d), (b, sk, hkv, d), (b, sk, hkv, d))]
+    dout = grid_values(rng, (b, sq, hq, d), -1.0, 1.0, e)
+
+    def loss(arrs, causal):
+        o, _, _ = run(lib, bf16(arrs[0]), bf16(arrs[1]), bf16(arrs[2]), causal, scale)
+        return float(np.sum(o.transpose(0, 2, 1, 3) * dout))
+
+    for causal in (False, True):
+        grads = oracle.attn_bwd(bf16(base[0]), bf16(base[1]), bf16(base[2]), bf16(dout), causal,
+                                scale, lib=lib)
+        for which in range(3):
+            for _ in range(4):
+                idx = tuple(int(rng.integers(0, n)) for n in base[which].shape)
+                plus = [a.copy() for a in base]
+                minus = [a.copy() for a in base]
+                plus[which][idx] += e
+                minus[which][idx] -= e
+                fd = (loss(plus, causal) - loss(minus, causal)) / (2 * e)
+                g = grads[which][idx]
+                assert abs(fd - g) <= 2e-4 + 2e-3 * abs(g), f"finite difference, input {which}"
+
+
+def pin_bwd_invariants(lib):
+    """Facts of the chain rule that need no second implementation: each row
+    of dS sums to 0, so the dK rows of a key/value head sum to 0; each row of
+    P sums to 1, so the dV rows sum to the sum of the group's dO rows; with
+    identical V rows dP is constant along a row, so dS = 0 and dQ = dK = 0."""
+    q, k, v = make_qkv(2, 4, 2, 23, 23, seed=46, d=8)
+    dout = make_qkv(2, 4, 2, 23, 23, seed=47, d=8)[0]
+    for causal in (False, True):
+        dq, dk, dv = oracle.attn_bwd(q, k, v, dout, causal, 0.5, lib=lib)
+        assert np.max(np.abs(dk.sum(axis=1))) < 1e-12, "dK rows do not sum to 0"
+        do = dout.double().numpy()
+        want = do.reshape(2, 23, 2, 2, 8).sum(axis=(1, 3))          # [b, kv head, d]
+        assert np.max(np.abs(dv.sum(axis=1) - want)) < 1e-12, "dV rows do not sum to sum dO"
+    rng = np.random.default_rng(48)
+    vrow = grid_values(rng, (2, 1, 2, 8))
+    v_same = bf16(np.broadcast_to(vrow, (2, 23, 2, 8)).copy())
+    dq, dk, dv = oracle.attn_bwd(q, k, v_same, dout, True, 0.5, lib=lib)
+    assert np.max(np.abs(dq)) < 1e-12 and np.max(np.abs(dk)) < 1e-12, "identical V rows"
+    # Causal, square: the last key is seen by the last row only.
+    _, _, p = run(lib, q, k, v, True, 0.5, want_p=True)
+    dq, dk, dv = oracle.attn_bwd(q, k, v, dout, True, 0.5, lib=lib)
+    want_v = sum(p[:, h, 22, 22][:, None] * do[:, 22, h] for h in (2, 3))   # kv head 1
+    assert np.max(np.abs(dv[:, 22, 1] - want_v)) < 1e-12, "causal last key"
+
+
 ALL_PINS = [
     pin_rows_sum_to_one, pin_identical_v_rows, pin_zero_query, pin_causal_row0,
     pin_causal_rectangular_is_square_suffix, pin_causal_single_query_sees_every_key,
@@ -380,6 +470,7 @@ ALL_PINS = [
     pin_key_shift, pin_value_affine, pin_key_permutation, pin_gqa_equals_repeated_mha,
     pin_torch_sdpa_f64, pin_golden_closed_forms, pin_row_subset,
     pin_varlen_matches_block_diagonal_sdpa, pin_varlen_sequences_are_independent,
+    pin_bwd_torch_autograd_f64, pin_bwd_finite_differences, pin_bwd_invariants,
 ]
 
 

@@ -113,6 +113,20 @@ MUTANTS = {
     "window_off_by_one": ("j < i + off - window_left)", "j < i + off - window_left + 1)"),
     "window_wrong_side": ("j < i + off - window_left)", "j > i + off - window_left)"),
     "bf16_decode_shift": ("((uint32_t)bits) << 16", "((uint32_t)bits) << 15"),
+    # backward
+    "bwd_dq_dropped_scale": ("dQb[(int64_t)i * qs + c] = scale * acc;",
+                             "dQb[(int64_t)i * qs + c] = acc;"),
+    "bwd_dk_dropped_scale": ("+= scale * acc_k;", "+= acc_k;"),
+    "bwd_D_sign": ("Prow[j] * (dProw[j] - Di);", "Prow[j] * (dProw[j] + Di);"),
+    "bwd_no_D": ("Prow[j] * (dProw[j] - Di);", "Prow[j] * dProw[j];"),
+    "bwd_dv_from_ds": ("acc_v += P[(int64_t)i * s_k + j]", "acc_v += dP[(int64_t)i * s_k + j]"),
+    "bwd_dk_from_p": ("acc_k += dP[(int64_t)i * s_k + j]", "acc_k += P[(int64_t)i * s_k + j]"),
+    "bwd_dp_with_k": ("dot += dOb[(int64_t)i * qs + c] * Vb[", "dot += dOb[(int64_t)i * qs + c] * Kb["),
+    "bwd_dq_with_v": ("acc += dSrow[j] * Kb[", "acc += dSrow[j] * Vb["),
+    "bwd_mask_off_by_one": ("if (causal && j > i + off) Prow[j]", "if (causal && j >= i + off) Prow[j]"),
+    "bwd_gqa_overwrites": ("dVb[(int64_t)j * ks + c] += acc_v;", "dVb[(int64_t)j * ks + c] = acc_v;"),
+    "bwd_D_from_first_key": ("for (int j = 0; j < s_k; ++j) Di += Prow[j] * dProw[j];",
+                             "for (int j = 0; j < 1; ++j) Di += Prow[j] * dProw[j];"),
 }
 
 
