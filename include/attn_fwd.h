@@ -100,6 +100,38 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
                     int window_left, float scale, void* stream);
 
 /*
+ * attn_fwd_varlen -- a packed batch of sequences of different lengths
+ * (the dynamic sequence-length support of the intelliparadigm.com AVO page,
+ * section 6): sequence b holds query rows cu_seqlens_q[b] ..
+ * cu_seqlens_q[b+1] - 1 and keys cu_seqlens_k[b] .. cu_seqlens_k[b+1] - 1
+ * of the packed tensors, and each sequence is its own attention problem
+ * (no query sees another sequence's keys; the causal mask and window are
+ * those of attn_fwd / attn_fwd_window with that sequence's s_q and s_k).
+ *
+ *   q    device, bf16 [total_q, h_q,  d] contiguous (read)
+ *   k    device, bf16 [total_k, h_kv, d] contiguous (read)
+ *   v    device, bf16 [total_k, h_kv, d] contiguous (read)
+ *   o    device, bf16 [total_q, h_q,  d] contiguous (written)
+ *   lse  device, fp32 [h_q, total_q]     contiguous (written)
+ *   cu_seqlens_q, cu_seqlens_k  device, int32 [batch + 1], non-decreasing,
+ *        starting at 0 and ending at total_q / total_k (4-byte aligned)
+ *   max_seqlen_q, max_seqlen_k  upper bounds of the sequences' lengths (the
+ *        launch has work items for max_seqlen_q rows per sequence)
+ *   causal, window_left  as attn_fwd / attn_fwd_window (window_left = -1:
+ *        none; a window needs causal = 1); causal needs s_q <= s_k per
+ *        sequence -- a row that sees no key gets O = 0, LSE = -inf
+ *
+ * The host cannot read cu_seqlens: sequences that break the rules above
+ * give unspecified values, but every access stays inside the packed
+ * tensors.  One launch; asynchronous; allocates nothing.
+ */
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cu_seqlens_q, const int* cu_seqlens_k, int batch,
+                    int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                    int h_q, int h_kv, int d, int causal, int window_left, float scale,
+                    void* stream);
+
+/*
  * attn_fwd_host -- the same forward on HOST buffers: copies q, k, v to the
  * device (cudaMemcpyAsync on `stream`), runs attn_fwd, copies o and lse back,
  * and returns without synchronising (the caller synchronises `stream` before

@@ -29,6 +29,11 @@ _I = ctypes.c_int
 _SIGNATURES = [
     ("attn_fwd", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]),
     ("attn_fwd_window", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float, _P]),
+    ("attn_fwd_varlen", _I, [_P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I, _I,
+                             _I, ctypes.c_float, _P]),
+    ("attn_bwd_workspace_bytes", ctypes.c_size_t, [_I, _I, _I]),
+    ("attn_bwd", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
+                      ctypes.c_float, _P, ctypes.c_size_t, _P]),
     ("attn_fwd_host", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
                            _P, ctypes.c_size_t, _P]),
     ("attn_fwd_host_workspace_bytes", ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
@@ -198,6 +203,78 @@ def attn_fwd_window(q, k, v, window_left: int, scale: float | None = None, o=Non
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_window")
     return o, lse
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_seqlen_k: int,
+                    causal: bool = False, scale: float | None = None, window_left: int = -1,
+                    o=None, lse=None, stream=None):
+    """Packed variable-length batch: q [total_q, h_q, 128], k/v
+    [total_k, h_kv, 128] (BF16, CUDA), cu_seqlens_* int32 CUDA tensors
+    [batch + 1].  Returns (o [total_q, h_q, 128] BF16, lse [h_q, total_q]
+    FP32)."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.bfloat16 or t.dim() != 3 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA bfloat16 [tokens, heads, dim]")
+    for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
+        if t.dtype != torch.int32 or t.dim() != 1 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA int32 vector")
+    total_q, h_q, d = q.shape
+    total_k, h_kv, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or dk != d:
+        raise ValueError("q, k, v shapes disagree")
+    batch = cu_seqlens_q.numel() - 1
+    if cu_seqlens_k.numel() != batch + 1 or batch < 1:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k need batch + 1 entries")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o, lse = _outputs(q, o, lse, (total_q, h_q, d), (h_q, total_q), stream)
+    rc = load_library().attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                        lse.data_ptr(), cu_seqlens_q.data_ptr(),
+                                        cu_seqlens_k.data_ptr(), batch, int(max_seqlen_q),
+                                        int(max_seqlen_k), total_q, total_k, h_q, h_kv, d,
+                                        int(bool(causal)), int(window_left), float(scale),
+                                        _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_varlen")
+    return o, lse
+
+
+def bwd_workspace_bytes(b, h_q, s_q) -> int:
+    return int(load_library().attn_bwd_workspace_bytes(b, h_q, s_q))
+
+
+def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = None,
+             window_left: int = -1, dq=None, dk=None, dv=None, workspace=None, stream=None):
+    """Gradients of the forward: (dq, dk, dv) BF16 in the layouts of q, k, v,
+    from the forward's o [b, s_q, h_q, 128] and lse [b, h_q, s_q] and the
+    incoming gradient dout (shaped like o).  Three launches on ``stream``."""
+    import torch
+    b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+    _check_out(o, "o", (b, s_q, h_q, d), torch.bfloat16, q.device)
+    _check_out(dout, "dout", (b, s_q, h_q, d), torch.bfloat16, q.device)
+    _check_out(lse, "lse", (b, h_q, s_q), torch.float32, q.device)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    dq, _ = _outputs(q, dq, None, (b, s_q, h_q, d), (1,), stream)
+    dk, _ = _outputs(k, dk, None, (b, s_k, h_kv, d), (1,), stream)
+    dv, _ = _outputs(v, dv, None, (b, s_k, h_kv, d), (1,), stream)
+    if workspace is None:
+        nbytes = bwd_workspace_bytes(b, h_q, s_q)
+        workspace = _alloc_on(stream, q.device,
+                              lambda: torch.empty(nbytes, dtype=torch.uint8, device=q.device))
+    rc = load_library().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                 dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
+                                 dv.data_ptr(), b, h_q, h_kv, s_q, s_k, d, int(bool(causal)),
+                                 int(window_left), float(scale), workspace.data_ptr(),
+                                 workspace.numel() * workspace.element_size(),
+                                 _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_bwd")
+    return dq, dk, dv
 
 
 def num_splits(b, h_q, h_kv, s_q, s_k, causal=False, d=128) -> int:

@@ -10,6 +10,7 @@
 #include <cstdlib>
 #include <mutex>
 
+#include "attn_bwd_kernel.cuh"
 #include "attn_fwd.h"
 #include "attn_fwd_kernel.cuh"
 #include "attn_merge.cuh"
@@ -56,12 +57,19 @@ int init_device(int dev, DeviceState** out) {
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
             return ATTN_ERR_CUDA;
-        if (cudaFuncSetAttribute(attn_fwd_sm100_kernel<false>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Layout::kAlloc) != cudaSuccess ||
-            cudaFuncSetAttribute(attn_fwd_sm100_kernel<true>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 Layout::kAlloc) != cudaSuccess)
+        const auto smem = cudaFuncAttributeMaxDynamicSharedMemorySize;
+        if (cudaFuncSetAttribute(attn_fwd_sm100_kernel<false, false>, smem, Layout::kAlloc) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(attn_fwd_sm100_kernel<true, false>, smem, Layout::kAlloc) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(attn_fwd_sm100_kernel<false, true>, smem, Layout::kAlloc) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(attn_fwd_sm100_kernel<true, true>, smem, Layout::kAlloc) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(bwd::dq::attn_bwd_dq_kernel, smem, bwd::dq::Smem::kAlloc) !=
+                cudaSuccess ||
+            cudaFuncSetAttribute(bwd::dkdv::attn_bwd_dkdv_kernel, smem,
+                                 bwd::dkdv::Smem::kAlloc) != cudaSuccess)
             return ATTN_ERR_CUDA;
         void* sp = nullptr;
         if (cudaGetSymbolAddress(&sp, g_status_word) != cudaSuccess) return ATTN_ERR_CUDA;
@@ -74,14 +82,16 @@ int init_device(int dev, DeviceState** out) {
 }
 
 // [batch, seq, heads, 128] BF16 as a 4-D tensor map {d, heads, seq, batch},
-// box {64, 1, 128, 1} (one 128-byte swizzled half of a 128-row tile).
-bool encode_map(CUtensorMap* m, const void* base, int heads, int seq, int batch) {
+// box {64, 1, box_rows, 1} (one 128-byte swizzled half of a box_rows-row
+// tile; 128 rows unless given).
+bool encode_map(CUtensorMap* m, const void* base, int heads, int seq, int batch,
+                unsigned box_rows = 128) {
     cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(heads),
                           static_cast<cuuint64_t>(seq), static_cast<cuuint64_t>(batch)};
     cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHeadDim) * 2,
                              static_cast<cuuint64_t>(heads) * kHeadDim * 2,
                              static_cast<cuuint64_t>(seq) * heads * kHeadDim * 2};
-    cuuint32_t box[4] = {64, 1, 128, 1};
+    cuuint32_t box[4] = {64, 1, box_rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -133,26 +143,44 @@ size_t split_workspace_bytes(int batch, int h_q, int s_q, int n_splits) {
            static_cast<size_t>(n_splits) * rows * 4;
 }
 
-// The forward launch shared by attn_fwd and attn_fwd_split (arguments
-// already validated).  o_part / lse_part null: O and LSE directly.
+// A packed variable-length batch: device cu_seqlens and the packed extents.
+struct Varlen {
+    const int* cu_q;
+    const int* cu_k;
+    int total_q, total_k;
+    int max_s_q, max_s_k;
+};
+
+// The forward launch shared by every forward entry point (arguments already
+// validated).  o_part / lse_part null: O and LSE directly.  varlen non-null:
+// a packed batch (batch = number of sequences; s_q, s_k unused).
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int batch,
                int h_q, int h_kv, int s_q, int s_k, int causal, int causal_offset, float scale,
                int n_splits, int kb_per_split, float* o_part, float* lse_part, void* stream,
-               int window_left = -1) {
+               int window_left = -1, const Varlen* varlen = nullptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
     DeviceState* st = nullptr;
     const int rc = init_device(dev, &st);
     if (rc != ATTN_OK) return rc;
 
+    // Packed tensors are one batch of total rows; the cursor adds each
+    // sequence's first row.
+    const int map_b = varlen ? 1 : batch;
+    const int map_sq = varlen ? varlen->total_q : s_q;
+    const int map_sk = varlen ? varlen->total_k : s_k;
+    if (varlen) {
+        s_q = varlen->max_s_q;
+        s_k = varlen->max_s_k;
+    }
     CUtensorMap tq, tk, tv, to;
-    if (!encode_map(&tq, q, h_q, s_q, batch) || !encode_map(&tk, k, h_kv, s_k, batch) ||
-        !encode_map(&tv, v, h_kv, s_k, batch))
+    if (!encode_map(&tq, q, h_q, map_sq, map_b) || !encode_map(&tk, k, h_kv, map_sk, map_b) ||
+        !encode_map(&tv, v, h_kv, map_sk, map_b))
         return ATTN_ERR_CUDA;
     // O is stored through a tensor map of the same shape as Q's (unused when
     // the launch writes FP32 partials instead).
     if (o != nullptr) {
-        if (!encode_map(&to, o, h_q, s_q, batch)) return ATTN_ERR_CUDA;
+        if (!encode_map(&to, o, h_q, map_sq, map_b)) return ATTN_ERR_CUDA;
     } else {
         to = tq;
     }
@@ -204,14 +232,23 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.status = st->status;
 
     p.window_left = window_left;
+    if (varlen) {
+        p.cu_q = varlen->cu_q;
+        p.cu_k = varlen->cu_k;
+        p.total_q = varlen->total_q;
+    }
 
     const int grid = p.num_tiles < st->num_sms ? p.num_tiles : st->num_sms;
-    if (window_left >= 0)
-        attn_fwd_sm100_kernel<true><<<grid, kThreads, Layout::kAlloc,
-                                      static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, to, p);
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const bool win = window_left >= 0;
+    if (!varlen && !win)
+        attn_fwd_sm100_kernel<false, false><<<grid, kThreads, Layout::kAlloc, cs>>>(tq, tk, tv, to, p);
+    else if (!varlen)
+        attn_fwd_sm100_kernel<true, false><<<grid, kThreads, Layout::kAlloc, cs>>>(tq, tk, tv, to, p);
+    else if (!win)
+        attn_fwd_sm100_kernel<false, true><<<grid, kThreads, Layout::kAlloc, cs>>>(tq, tk, tv, to, p);
     else
-        attn_fwd_sm100_kernel<false><<<grid, kThreads, Layout::kAlloc,
-                                       static_cast<cudaStream_t>(stream)>>>(tq, tk, tv, to, p);
+        attn_fwd_sm100_kernel<true, true><<<grid, kThreads, Layout::kAlloc, cs>>>(tq, tk, tv, to, p);
     g_last_launches = 1;
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     return ATTN_OK;
@@ -272,6 +309,120 @@ extern "C" int attn_fwd_window(const void* q, const void* k, const void* v, void
     const int w = window_left >= s_k ? -1 : window_left;
     return launch_fwd(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, 1, s_k - s_q, scale, 1, n_kb,
                       nullptr, nullptr, stream, w);
+}
+
+extern "C" int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                               const int* cu_seqlens_q, const int* cu_seqlens_k, int batch,
+                               int max_seqlen_q, int max_seqlen_k, int total_q, int total_k,
+                               int h_q, int h_kv, int d, int causal, int window_left,
+                               float scale, void* stream) {
+    if (!cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID;
+    // The packed tensors are validated as one batch of total rows.
+    int rc = validate(q, k, v, o, lse, 1, h_q, h_kv, total_q, total_k, d, 0, scale);
+    if (rc != ATTN_OK) return rc;
+    if (batch <= 0 || max_seqlen_q <= 0 || max_seqlen_k <= 0) return ATTN_ERR_INVALID;
+    if (causal != 0 && causal != 1) return ATTN_ERR_INVALID;
+    if (window_left < -1 || (window_left >= 0 && !causal)) return ATTN_ERR_INVALID;
+    if (!aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4)) return ATTN_ERR_ALIGN;
+    const long long n_qb = (max_seqlen_q + kBlockM - 1) / kBlockM;
+    if (static_cast<long long>(batch) * h_q * ((n_qb + 1) / 2) > 0x7fffffffLL)
+        return ATTN_ERR_INVALID;
+    Varlen vl{cu_seqlens_q, cu_seqlens_k, total_q, total_k, max_seqlen_q, max_seqlen_k};
+    const int n_kb = (max_seqlen_k + kBlockN - 1) / kBlockN;
+    const int w = (window_left >= max_seqlen_k) ? -1 : window_left;
+    return launch_fwd(q, k, v, o, lse, batch, h_q, h_kv, max_seqlen_q, max_seqlen_k, causal, 0,
+                      scale, 1, n_kb, nullptr, nullptr, stream, w, &vl);
+}
+
+extern "C" size_t attn_bwd_workspace_bytes(int batch, int h_q, int s_q) {
+    if (batch <= 0 || h_q <= 0 || s_q <= 0) return 0;
+    const size_t pad = static_cast<size_t>((s_q + kBlockM - 1) / kBlockM) * kBlockM;
+    return 2 * static_cast<size_t>(batch) * h_q * pad * sizeof(float);
+}
+
+extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                        const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                        int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal,
+                        int window_left, float scale, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+    int rc = validate(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale);
+    if (rc != ATTN_OK) return rc;
+    if (!dout || !dq || !dk || !dv || !workspace) return ATTN_ERR_INVALID;
+    if (window_left < -1 || (window_left >= 0 && !causal)) return ATTN_ERR_INVALID;
+    if (!aligned(dout, 16) || !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) ||
+        !aligned(workspace, 256))
+        return ATTN_ERR_ALIGN;
+    if (workspace_bytes < attn_bwd_workspace_bytes(batch, h_q, s_q)) return ATTN_ERR_INVALID;
+    const long long n_qb64 = (s_q + bwd::kBlockQ - 1) / bwd::kBlockQ;
+    const long long n_kb = (s_k + kBlockN - 1) / kBlockN;
+    if (static_cast<long long>(batch) * h_q * n_qb64 > 0x7fffffffLL ||
+        static_cast<long long>(batch) * h_kv * n_kb > 0x7fffffffLL)
+        return ATTN_ERR_INVALID;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    DeviceState* st = nullptr;
+    rc = init_device(dev, &st);
+    if (rc != ATTN_OK) return rc;
+    const cudaStream_t cs = static_cast<cudaStream_t>(stream);
+
+    bwd::BwdParams p{};
+    p.batch = batch;
+    p.h_q = h_q;
+    p.h_kv = h_kv;
+    p.s_q = s_q;
+    p.s_k = s_k;
+    p.group = h_q / h_kv;
+    p.n_qb = (s_q + kBlockM - 1) / kBlockM;
+    p.n_kb = static_cast<int>(n_kb);
+    p.n_qb64 = static_cast<int>(n_qb64);
+    p.s_q_pad = p.n_qb * kBlockM;
+    p.causal = causal;
+    p.causal_offset = s_k - s_q;
+    p.window_left = (window_left >= s_k) ? -1 : window_left;
+    p.div_h_q = FastDiv::make(static_cast<uint32_t>(h_q));
+    p.div_h_kv = FastDiv::make(static_cast<uint32_t>(h_kv));
+    p.scale = scale;
+    p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
+    float* Lw = static_cast<float*>(workspace);
+    float* Dw = Lw + static_cast<size_t>(batch) * h_q * p.s_q_pad;
+    p.L = Lw;
+    p.D = Dw;
+    p.timeout_ns = g_timeout_ns;
+    p.status = st->status;
+
+    // 1. D = rowsum(dO * O) and L = LSE log2(e), padded per head.
+    bwd::PrepParams a{static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout),
+                      lse, Lw, Dw, batch, h_q, s_q, p.s_q_pad};
+    const size_t rows = static_cast<size_t>(batch) * h_q * p.s_q_pad;
+    size_t blocks = (rows + bwd::kPrepThreads / 32 - 1) / (bwd::kPrepThreads / 32);
+    const size_t cap = static_cast<size_t>(st->num_sms) * 16;
+    if (blocks > cap) blocks = cap;
+    bwd::attn_bwd_prep_kernel<<<static_cast<unsigned>(blocks), bwd::kPrepThreads, 0, cs>>>(a);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+    CUtensorMap tq, tk, tv, tdo, tdq, tq64, tdo64, tdk, tdv;
+    if (!encode_map(&tq, q, h_q, s_q, batch) || !encode_map(&tk, k, h_kv, s_k, batch) ||
+        !encode_map(&tv, v, h_kv, s_k, batch) || !encode_map(&tdo, dout, h_q, s_q, batch) ||
+        !encode_map(&tdq, dq, h_q, s_q, batch) || !encode_map(&tq64, q, h_q, s_q, batch, 64) ||
+        !encode_map(&tdo64, dout, h_q, s_q, batch, 64) ||
+        !encode_map(&tdk, dk, h_kv, s_k, batch) || !encode_map(&tdv, dv, h_kv, s_k, batch))
+        return ATTN_ERR_CUDA;
+
+    // 2. dK, dV: one item per (key block, batch, key/value head).
+    p.num_items = batch * h_kv * p.n_kb;
+    int grid = p.num_items < st->num_sms ? p.num_items : st->num_sms;
+    bwd::dkdv::attn_bwd_dkdv_kernel<<<grid, bwd::kThreads, bwd::dkdv::Smem::kAlloc, cs>>>(
+        tq64, tk, tv, tdo64, tdk, tdv, p);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+
+    // 3. dQ: one item per (query block, batch, query head).
+    p.num_items = batch * h_q * p.n_qb;
+    grid = p.num_items < st->num_sms ? p.num_items : st->num_sms;
+    bwd::dq::attn_bwd_dq_kernel<<<grid, bwd::kThreads, bwd::dq::Smem::kAlloc, cs>>>(tq, tk, tv,
+                                                                                     tdo, tdq, p);
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+    g_last_launches = 3;
+    return ATTN_OK;
 }
 
 extern "C" int attn_fwd_num_splits(int batch, int h_q, int h_kv, int s_q, int s_k, int d,

@@ -85,6 +85,12 @@ struct FwdParams {
     unsigned long long timeout_ns;
     unsigned int* status;
     int window_left;  // sliding window (windowed kernel only): keys before the diagonal
+    // Packed variable-length batch (varlen kernel only): sequence b holds
+    // packed query rows cu_q[b] .. cu_q[b+1] - 1 and keys cu_k[b] ..
+    // cu_k[b+1] - 1; O is [total_q][h_q][128], LSE [h_q][total_q].
+    const int* cu_q;
+    const int* cu_k;
+    int total_q;
 };
 
 // ------------------------------------------------------------------ waits

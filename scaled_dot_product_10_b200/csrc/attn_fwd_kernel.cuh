@@ -91,7 +91,11 @@ constexpr uint32_t kRegsControl = 72;
 // different key intervals: iteration t of the pair's K/V stream is key block
 // kb0 + t; block 0 visits iterations 0 .. n[0] - 1 and block 1 iterations
 // st1 .. st1 + n[1] - 1 (its window starts st1 key blocks later).
-template <bool kWindow>
+//
+// In a packed variable-length batch (kVarlen) "batch" b is sequence b: its
+// query rows are cu_q[b] .. cu_q[b+1] - 1 and its keys cu_k[b] .. cu_k[b+1]
+// - 1 of the packed tensors, and the pairs past its own length have no work.
+template <bool kWindow, bool kVarlen>
 struct PairCursor {
     int round;  // rounds of gridDim.x items dealt so far
     int t;
@@ -99,12 +103,15 @@ struct PairCursor {
     int split, kb0;  // key range of the item: key blocks kb0 .. kb0 + n[i] - 1
     int n[2];        // key/value blocks each query block of the pair visits (0: none)
     int st1;         // kWindow: first iteration of block 1 (0 otherwise)
+    // kVarlen: the sequence's first packed query row and key, its lengths
+    // and its causal offset s_k - s_q.
+    int q_row0, k_row0, s_q, s_k, off;
 
     __device__ __forceinline__ void decode(const FwdParams& p) {
         const int u = p.div_splits.div(t);
         split = t - u * p.n_splits;
         kb0 = split * p.kb_per_split;
-        const int kb_end = min(p.n_kb, kb0 + p.kb_per_split);
+        int kb_end = min(p.n_kb, kb0 + p.kb_per_split);
         const int G = p.units_per_section;
         const int sec = p.div_section.div(u);
         const int r = u - sec * G * p.group * p.n_pairs;
@@ -120,27 +127,46 @@ struct PairCursor {
         g = unit - b * p.h_kv;
         h = g * p.group + h_local;
         qb0 = 2 * pair;
+        int sq = p.s_q, nqb = p.n_qb, coff = p.causal_offset;
+        if constexpr (kVarlen) {
+            // No key ranges here (kb0 = 0): the sequence's own extents.
+            q_row0 = __ldg(p.cu_q + b);
+            s_q = __ldg(p.cu_q + b + 1) - q_row0;
+            k_row0 = __ldg(p.cu_k + b);
+            s_k = __ldg(p.cu_k + b + 1) - k_row0;
+            off = s_k - s_q;
+            sq = s_q;
+            nqb = max(0, (s_q + kBlockM - 1) >> 7);
+            coff = off;
+            kb_end = max(0, (s_k + kBlockN - 1) >> 7);
+        }
         // Causal: the last row of block qb, min(128 qb + 127, s_q - 1), sees
         // keys up to row + causal_offset (s_k - s_q, or a key shard's own
         // diagonal, which may be negative: floor division by the shift).
         static_assert(kBlockN == 128, "the shift below divides by kBlockN");
-        const int last0 = (min(qb0 * kBlockM + kBlockM - 1, p.s_q - 1) + p.causal_offset) >> 7;
-        const int last1 = (min(qb0 * kBlockM + 2 * kBlockM - 1, p.s_q - 1) + p.causal_offset) >> 7;
+        const int last0 = (min(qb0 * kBlockM + kBlockM - 1, sq - 1) + coff) >> 7;
+        const int last1 = (min(qb0 * kBlockM + 2 * kBlockM - 1, sq - 1) + coff) >> 7;
         const int vis0 = p.causal ? min(kb_end, last0 + 1) : kb_end;
-        const int vis1 = (qb0 + 1 < p.n_qb) ? (p.causal ? min(kb_end, last1 + 1) : kb_end) : 0;
+        const int vis1 = (qb0 + 1 < nqb) ? (p.causal ? min(kb_end, last1 + 1) : kb_end) : 0;
         n[0] = max(0, vis0 - kb0);
         n[1] = max(0, vis1 - kb0);
+        if constexpr (kVarlen) {
+            if (qb0 >= nqb) n[0] = 0;  // the pair lies past this sequence
+        }
         if constexpr (kWindow) {
             // Causal with a window of window_left keys before the diagonal
             // (no key ranges): row r sees keys r + causal_offset -
             // window_left .. r + causal_offset, so a block starts at the key
             // block of its first row's lower bound.
-            const int lo0 = max(0, (qb0 * kBlockM + p.causal_offset - p.window_left) >> 7);
-            const int lo1 = max(0, ((qb0 + 1) * kBlockM + p.causal_offset - p.window_left) >> 7);
+            const int lo0 = max(0, (qb0 * kBlockM + coff - p.window_left) >> 7);
+            const int lo1 = max(0, ((qb0 + 1) * kBlockM + coff - p.window_left) >> 7);
             kb0 = lo0;
-            n[0] = vis0 - lo0;
+            n[0] = max(0, vis0 - lo0);
             st1 = lo1 - lo0;
-            n[1] = (qb0 + 1 < p.n_qb) ? vis1 - lo1 : 0;
+            n[1] = (qb0 + 1 < nqb) ? max(0, vis1 - lo1) : 0;
+            if constexpr (kVarlen) {
+                if (qb0 >= nqb) n[0] = 0;
+            }
         } else {
             st1 = 0;
         }
@@ -239,7 +265,7 @@ __device__ __forceinline__ void exp_row(const float (&s)[128], uint64_t c2x2, ui
 
 // ------------------------------------------------------------------ softmax
 // One softmax warpgroup: thread r owns query row r of its block (TMEM lane r).
-template <bool kWindow>
+template <bool kWindow, bool kVarlen>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorMap* tm_o,
                                              const WaitCtx& wc, uint32_t tmem, uint32_t sP,
                                              uint32_t bars, int wg, int warp_in_wg, int lane) {
@@ -270,7 +296,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
     uint32_t cnt = 0;     // S blocks this warpgroup has processed (all pairs)
     uint32_t stored = 0;  // O tiles this warpgroup has stored through TMA
     uint32_t rounds = 0;  // alternation rounds before this pair
-    PairCursor<kWindow> c;
+    PairCursor<kWindow, kVarlen> c;
     c.start(p);
     for (; c.valid(p); c.next(p)) {
         const int n = c.n[wg];
@@ -309,21 +335,25 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
             if (lane == 0) ptx::mbar_arrive(b_sfree);
 
             const int kv0 = (c.kb0 + t0 + j) * kBlockN;
-            const bool diag = p.causal && (kv0 + kBlockN - 1 > qb * kBlockM + p.causal_offset);
-            bool masked = diag || kv0 + kBlockN > p.s_k;
+            int seq_k = p.s_k, coff = p.causal_offset;
+            if constexpr (kVarlen) {
+                seq_k = c.s_k;
+                coff = c.off;
+            }
+            const bool diag = p.causal && (kv0 + kBlockN - 1 > qb * kBlockM + coff);
+            bool masked = diag || kv0 + kBlockN > seq_k;
             if constexpr (kWindow) {
                 // keys before the last row's window start
-                masked = masked ||
-                         kv0 < qb * kBlockM + kBlockM - 1 + p.causal_offset - p.window_left;
+                masked = masked || kv0 < qb * kBlockM + kBlockM - 1 + coff - p.window_left;
             }
             if (masked) {
-                const int lim_tail = p.s_k - kv0;                           // keys >= s_k
+                const int lim_tail = seq_k - kv0;                           // keys >= s_k
                 // keys past row + s_k - s_q
-                const int lim_causal = p.causal ? row + p.causal_offset - kv0 + 1 : kBlockN;
+                const int lim_causal = p.causal ? row + coff - kv0 + 1 : kBlockN;
                 const int lim = min(lim_tail, lim_causal);
                 if constexpr (kWindow) {
                     // and keys before row + s_k - s_q - window_left
-                    const int lo = row + p.causal_offset - p.window_left - kv0;
+                    const int lo = row + coff - p.window_left - kv0;
 #pragma unroll
                     for (int k = 0; k < 128; ++k)
                         if (k >= lim || k < lo) s[k] = -CUDART_INF_F;
@@ -413,7 +443,12 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
                 // range), LSE in natural log.
                 if (!wait_bar_warp(b_ofull, cnt & 1, wc)) return;
                 ptx::tc_fence_after();
-                const float inv_l = 1.f / l_run;
+                float inv_l = 1.f / l_run;
+                if constexpr (kVarlen) {
+                    // A causal row of a sequence with fewer keys than
+                    // queries may see no key: O = 0 (LSE = -inf).
+                    inv_l = l_run > 0.f ? inv_l : 0.f;
+                }
                 const uint64_t il2 = ptx::f2_pack(inv_l, inv_l);
                 const float lse_row = (m_ref * c2 + __log2f(l_run)) * 0.69314718055994531f;
                 const size_t row_id = (static_cast<size_t>(c.b) * p.h_q + c.h) * p.s_q + row;
@@ -454,7 +489,20 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
                     // BF16 O rows go to this block's P buffer (free: the last
                     // P V has completed) in the tile layout TMA reads, and
                     // one thread stores the tile with two TMA copies (rows
-                    // past s_q are clipped by the tensor map).
+                    // past s_q are clipped by the tensor map).  In a packed
+                    // batch a sequence's last, partial tile is written row
+                    // by row instead (a tile store would overwrite the next
+                    // sequence's rows); every row stays inside the packed
+                    // tensor even if cu_seqlens are inconsistent.
+                    bool tma_tile = true;
+                    bool row_ok = true;
+                    __nv_bfloat16* orow = nullptr;
+                    if constexpr (kVarlen) {
+                        tma_tile = (qb + 1) * kBlockM <= c.s_q &&
+                                   c.q_row0 + (qb + 1) * kBlockM <= p.total_q;
+                        row_ok = row < c.s_q && c.q_row0 + row < p.total_q;
+                        orow = p.o + (static_cast<size_t>(c.q_row0 + row) * p.h_q + c.h) * kHeadDim;
+                    }
 #pragma unroll
                     for (int q = 0; q < 4; ++q) {
                         uint32_t ov[32];
@@ -470,12 +518,19 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
                             ptx::f2_unpack(v, lo, hi);
                             w[k] = ptx::pack_bf16x2(lo, hi);
                         }
+                        if (tma_tile) {
 #pragma unroll
-                        for (int k = 0; k < 4; ++k) {
-                            const int cc = 4 * q + k;
-                            ptx::st_shared_v4(
-                                p_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ p_xor) << 4),
-                                w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                            for (int k = 0; k < 4; ++k) {
+                                const int cc = 4 * q + k;
+                                ptx::st_shared_v4(
+                                    p_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ p_xor) << 4),
+                                    w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                            }
+                        } else if (row_ok) {
+#pragma unroll
+                            for (int k = 0; k < 4; ++k)
+                                reinterpret_cast<uint4*>(orow)[4 * q + k] =
+                                    make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
                         }
                     }
                     ptx::tc_fence_before();
@@ -488,16 +543,29 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
                     if (lane == 0) ptx::mbar_arrive(b_ostaged);
                     if (r == 0) {
                         if (!wait_bar(b_ostaged, stored & 1, wc)) return;
-                        const uint32_t tile = sP + wg * kTileBytes;
-                        ptx::tma_store_4d(tm_o, tile, 0, c.h, qb * kBlockM, c.b);
-                        ptx::tma_store_4d(tm_o, tile + kHalfTileBytes, 64, c.h, qb * kBlockM, c.b);
-                        ptx::bulk_commit_group();
-                        ptx::bulk_wait_group_read0();
+                        if (tma_tile) {
+                            const uint32_t tile = sP + wg * kTileBytes;
+                            int row0 = qb * kBlockM, bc = c.b;
+                            if constexpr (kVarlen) {
+                                row0 += c.q_row0;  // packed rows, batch extent 1
+                                bc = 0;
+                            }
+                            ptx::tma_store_4d(tm_o, tile, 0, c.h, row0, bc);
+                            ptx::tma_store_4d(tm_o, tile + kHalfTileBytes, 64, c.h, row0, bc);
+                            ptx::bulk_commit_group();
+                            ptx::bulk_wait_group_read0();
+                        }
                         ptx::mbar_arrive(b_ostored);
                     }
                     if (!wait_bar_warp(b_ostored, stored & 1, wc)) return;
                     ++stored;
-                    if (row < p.s_q) p.lse[row_id] = lse_row;
+                    if constexpr (kVarlen) {
+                        // LSE [h_q][total_q]
+                        if (row_ok)
+                            p.lse[static_cast<size_t>(c.h) * p.total_q + c.q_row0 + row] = lse_row;
+                    } else {
+                        if (row < p.s_q) p.lse[row_id] = lse_row;
+                    }
                 }
             }
         }
@@ -506,7 +574,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
 }
 
 // ------------------------------------------------------------------ kernel
-template <bool kWindow>
+template <bool kWindow, bool kVarlen>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
@@ -582,14 +650,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t q_loads[2] = {0, 0};
             bool ok = true;
             auto load_tile = [&](const CUtensorMap* tm, uint32_t dst, uint32_t full,
-                                 const PairCursor<kWindow>& c,
+                                 const PairCursor<kWindow, kVarlen>& c,
                                  int j) {
                 ptx::mbar_arrive_expect_tx(full, kTileBytes);
-                const int key0 = (c.kb0 + j) * kBlockN;
-                ptx::tma_load_4d(dst, tm, full, 0, c.g, key0, c.b, pol_kv);
-                ptx::tma_load_4d(dst + kHalfTileBytes, tm, full, 64, c.g, key0, c.b, pol_kv);
+                int key0 = (c.kb0 + j) * kBlockN, bc = c.b;
+                if constexpr (kVarlen) {
+                    key0 += c.k_row0;  // packed keys, batch extent 1
+                    bc = 0;
+                }
+                ptx::tma_load_4d(dst, tm, full, 0, c.g, key0, bc, pol_kv);
+                ptx::tma_load_4d(dst + kHalfTileBytes, tm, full, 64, c.g, key0, bc, pol_kv);
             };
-            auto load_k = [&](const PairCursor<kWindow>& c, int j) -> bool {
+            auto load_k = [&](const PairCursor<kWindow, kVarlen>& c, int j) -> bool {
                 const int slot = k_loads % kKStages;
                 if (!wait_bar(bar(L::bKEmpty + slot), ((k_loads / kKStages) & 1) ^ 1, wc))
                     return false;
@@ -597,7 +669,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++k_loads;
                 return true;
             };
-            auto load_v = [&](const PairCursor<kWindow>& c, int j) -> bool {
+            auto load_v = [&](const PairCursor<kWindow, kVarlen>& c, int j) -> bool {
                 const int slot = v_loads % kVStages;
                 if (!wait_bar(bar(L::bVEmpty + slot), ((v_loads / kVStages) & 1) ^ 1, wc))
                     return false;
@@ -605,7 +677,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++v_loads;
                 return true;
             };
-            PairCursor<kWindow> c;
+            PairCursor<kWindow, kVarlen> c;
             c.start(p);
             for (; ok && c.valid(p); c.next(p)) {
 #pragma unroll
@@ -616,11 +688,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         continue;
                     }
                     const uint32_t dst = sQ + i * kTileBytes;
-                    const int row0 = (c.qb0 + i) * kBlockM;
+                    int row0 = (c.qb0 + i) * kBlockM, bc = c.b;
+                    if constexpr (kVarlen) {
+                        row0 += c.q_row0;
+                        bc = 0;
+                    }
                     ptx::mbar_arrive_expect_tx(bar(L::bQFull + i), kTileBytes);
-                    ptx::tma_load_4d(dst, &tm_q, bar(L::bQFull + i), 0, c.h, row0, c.b, pol_q);
+                    ptx::tma_load_4d(dst, &tm_q, bar(L::bQFull + i), 0, c.h, row0, bc, pol_q);
                     ptx::tma_load_4d(dst + kHalfTileBytes, &tm_q, bar(L::bQFull + i), 64, c.h,
-                                     row0, c.b, pol_q);
+                                     row0, bc, pol_q);
                     ++q_loads[i];
                 }
                 // Issue order = the MMA warp's consumption order:
@@ -727,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ++pv_cnt;
                 return true;
             };
-            PairCursor<kWindow> c;
+            PairCursor<kWindow, kVarlen> c;
             c.start(p);
             for (; ok && c.valid(p); c.next(p)) {
                 const int n = c.iters();
@@ -790,7 +866,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp < 8) {
         ptx::reg_alloc<kRegsSoftmax>();
-        softmax_role<kWindow>(p, &tm_o, wc, tmem, sP, bars, warp >> 2, warp & 3, lane);
+        softmax_role<kWindow, kVarlen>(p, &tm_o, wc, tmem, sP, bars, warp >> 2, warp & 3, lane);
     } else {
         ptx::reg_dealloc<kRegsControl>();  // idle warps of the control warpgroup
     }

@@ -213,3 +213,59 @@ def test_window_entry_validation(lib):
     assert f(A + 8, *ok[1:], 10, 0.088, None) == attn.ATTN_ERR_ALIGN
     if not torch.cuda.is_available():
         assert f(*ok, 10, 0.088, None) == attn.ATTN_ERR_CUDA
+
+
+def test_varlen_entry_validation(lib):
+    f = lib.attn_fwd_varlen
+    # q, k, v, o, lse, cu_q, cu_k, batch, max_q, max_k, total_q, total_k, h_q, h_kv, d,
+    # causal, window_left, scale
+    ok = [A, A, A, A, A, A, A, 2, 300, 300, 400, 400, 4, 2, 128, 1, -1, 0.088, None]
+
+    def call_with(**kw):
+        names = ["q", "k", "v", "o", "lse", "cq", "ck", "b", "mq", "mk", "tq", "tk", "hq",
+                 "hkv", "d", "causal", "w", "scale", "stream"]
+        a = dict(zip(names, ok))
+        a.update(kw)
+        return f(*[a[n] for n in names])
+
+    assert call_with(cq=0) == attn.ATTN_ERR_INVALID
+    assert call_with(ck=0) == attn.ATTN_ERR_INVALID
+    assert call_with(b=0) == attn.ATTN_ERR_INVALID
+    assert call_with(mq=0) == attn.ATTN_ERR_INVALID
+    assert call_with(tq=0) == attn.ATTN_ERR_INVALID
+    assert call_with(hq=3) == attn.ATTN_ERR_INVALID
+    assert call_with(d=64) == attn.ATTN_ERR_UNSUPPORTED
+    assert call_with(causal=2) == attn.ATTN_ERR_INVALID
+    assert call_with(w=-2) == attn.ATTN_ERR_INVALID
+    assert call_with(causal=0, w=5) == attn.ATTN_ERR_INVALID
+    assert call_with(cq=A + 2) == attn.ATTN_ERR_ALIGN
+    assert call_with(q=A + 8) == attn.ATTN_ERR_ALIGN
+    if not torch.cuda.is_available():
+        assert call_with() == attn.ATTN_ERR_CUDA
+
+
+def test_bwd_entry_validation(lib):
+    f = lib.attn_bwd
+    need = lib.attn_bwd_workspace_bytes(1, 2, 256)
+    assert need == 2 * 1 * 2 * 256 * 4
+    assert lib.attn_bwd_workspace_bytes(0, 2, 256) == 0
+    base = [A, A, A, A, A, A, A, A, A, 1, 2, 2, 256, 256, 128, 1, -1, 0.088, A, need, None]
+
+    def call_with(i, val):
+        a = list(base)
+        a[i] = val
+        return f(*a)
+
+    for i in range(9):          # any null pointer
+        assert call_with(i, 0) == attn.ATTN_ERR_INVALID
+    assert call_with(18, 0) == attn.ATTN_ERR_INVALID          # workspace
+    assert call_with(19, need - 1) == attn.ATTN_ERR_INVALID   # too small
+    assert call_with(18, A + 16) == attn.ATTN_ERR_ALIGN       # workspace alignment
+    assert call_with(6, A + 8) == attn.ATTN_ERR_ALIGN         # dq
+    assert call_with(14, 64) == attn.ATTN_ERR_UNSUPPORTED     # d
+    assert call_with(16, -2) == attn.ATTN_ERR_INVALID         # window
+    a = list(base)
+    a[15], a[16] = 0, 5                                       # window without causal
+    assert f(*a) == attn.ATTN_ERR_INVALID
+    if not torch.cuda.is_available():
+        assert f(*base) == attn.ATTN_ERR_CUDA
