@@ -58,6 +58,17 @@ def load(path: str | None = None):
         ctypes.c_int, ctypes.c_int, ctypes.c_double,
         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
     ]
+    lib.oracle_attn_fwd_fp8_f64.restype = ctypes.c_int
+    lib.oracle_attn_fwd_fp8_f64.argtypes = [
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ctypes.c_double, ctypes.c_double, ctypes.c_double,
+        ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        ctypes.c_int, ctypes.c_int, ctypes.c_double,
+        ctypes.c_void_p, ctypes.c_int,
+        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+    ]
+    lib.oracle_e4m3_to_double.restype = ctypes.c_double
+    lib.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
     lib.oracle_num_threads.restype = ctypes.c_int
     if path is None:
         _lib = lib
@@ -185,3 +196,49 @@ def attn_bwd(q, k, v, dout, causal: bool, scale: float, window_left: int = -1, l
     if rc != 0:
         raise ValueError(f"oracle rejected its arguments (code {rc})")
     return dq, dk, dv
+
+
+def _as_bytes(x) -> np.ndarray:
+    """Accept a torch float8_e4m3fn / uint8 tensor or a numpy uint8 array."""
+    if isinstance(x, np.ndarray):
+        if x.dtype != np.uint8:
+            raise TypeError("numpy FP8 inputs must be uint8 arrays of e4m3 bits")
+        return np.ascontiguousarray(x)
+    import torch
+    t = x.detach().cpu().contiguous()
+    if t.dtype not in (torch.float8_e4m3fn, torch.uint8):
+        raise TypeError("torch FP8 inputs must be float8_e4m3fn (or uint8 bits)")
+    return np.ascontiguousarray(t.view(torch.uint8).numpy())
+
+
+def e4m3_to_double(bits: int, lib=None) -> float:
+    return float((lib or load()).oracle_e4m3_to_double(int(bits)))
+
+
+def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, causal: bool,
+                 scale: float, rows=None, lib=None, window_left: int = -1):
+    """The forward on FP8 E4M3 inputs with per-tensor scales (input values are
+    scale * e4m3 value).  Shapes and outputs as :func:`attn_fwd`."""
+    qb, kb, vb = _as_bytes(q), _as_bytes(k), _as_bytes(v)
+    batch, s_q, h_q, d = qb.shape
+    bk, s_k, h_kv, dk = kb.shape
+    if vb.shape != kb.shape or bk != batch or dk != d:
+        raise ValueError("shape mismatch between q, k and v")
+    if rows is None:
+        n_rows, rows_arr = s_q, None
+    else:
+        rows_arr = np.ascontiguousarray(np.asarray(rows, dtype=np.int32))
+        if rows_arr.ndim != 3 or rows_arr.shape[:2] != (batch, h_q):
+            raise ValueError("rows must have shape [batch, h_q, n_rows]")
+        n_rows = rows_arr.shape[2]
+    o = np.zeros((batch, h_q, n_rows, d), dtype=np.float64)
+    lse = np.zeros((batch, h_q, n_rows), dtype=np.float64)
+    lib = lib or load()
+    rc = lib.oracle_attn_fwd_fp8_f64(
+        qb.ctypes.data, kb.ctypes.data, vb.ctypes.data, float(q_scale), float(k_scale),
+        float(v_scale), batch, h_q, h_kv, s_q, s_k, d, int(bool(causal)), int(window_left),
+        float(scale), None if rows_arr is None else rows_arr.ctypes.data, n_rows,
+        o.ctypes.data, lse.ctypes.data, None)
+    if rc != 0:
+        raise ValueError(f"oracle rejected its arguments (code {rc})")
+    return o, lse

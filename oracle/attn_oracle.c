@@ -136,6 +136,26 @@ static void attend_rows(const double *Q, const double *K, const double *V,
     }
 }
 
+/* FP8 E4M3 (the "e4m3fn" variant): 1 sign bit, 4 exponent bits with bias 7,
+ * 3 mantissa bits; exponent 0 encodes subnormals m * 2^-9; there are no
+ * infinities, and S.1111.111 is NaN.  Decoded exactly into a double. */
+static double e4m3_to_double(uint8_t bits)
+{
+    const int sign = bits >> 7, e = (bits >> 3) & 15, m = bits & 7;
+    double mag;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) mag = ldexp((double)m, -9);
+    else mag = ldexp(1.0 + m / 8.0, e - 7);
+    return sign ? -mag : mag;
+}
+
+double oracle_e4m3_to_double(uint8_t bits) { return e4m3_to_double(bits); }
+
+static int forward_on_doubles(double *Q, double *K, double *V, int batch, int h_q, int h_kv,
+                              int s_q, int s_k, int d, int causal, int window_left,
+                              double scale, const int32_t *rows, int n_rows, double *o,
+                              double *lse, double *p);
+
 int oracle_attn_fwd_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
                         int batch, int h_q, int h_kv, int s_q, int s_k, int d,
                         int causal, int window_left, double scale,
@@ -159,7 +179,55 @@ int oracle_attn_fwd_f64(const uint16_t *q, const uint16_t *k, const uint16_t *v,
     double *K = decode_bf16(k, (int64_t)batch * s_k * h_kv * d);
     double *V = decode_bf16(v, (int64_t)batch * s_k * h_kv * d);
     if (!Q || !K || !V) { free(Q); free(K); free(V); return -7; }
+    return forward_on_doubles(Q, K, V, batch, h_q, h_kv, s_q, s_k, d, causal, window_left,
+                              scale, rows, n_rows, o, lse, p);
+}
 
+/*
+ * The forward on FP8 E4M3 inputs with per-tensor scales: the inputs are the
+ * values Q = q_scale * e4m3(q), K = k_scale * e4m3(k), V = v_scale * e4m3(v),
+ * decoded exactly into doubles; everything after that is the forward above
+ * (the pages' low-precision GEMM inputs with higher-precision softmax: the
+ * bjdmk.com.cn survey page, section 3; the rkmt.cn page, section 3.1.1).
+ * Layouts as oracle_attn_fwd_f64 with one byte per input element.
+ */
+int oracle_attn_fwd_fp8_f64(const uint8_t *q, const uint8_t *k, const uint8_t *v,
+                            double q_scale, double k_scale, double v_scale,
+                            int batch, int h_q, int h_kv, int s_q, int s_k, int d,
+                            int causal, int window_left, double scale,
+                            const int32_t *rows, int n_rows,
+                            double *o, double *lse, double *p)
+{
+    if (!q || !k || !v || !o || !lse) return -1;
+    if (batch <= 0 || h_q <= 0 || h_kv <= 0 || s_q <= 0 || s_k <= 0 || d <= 0) return -2;
+    if (h_q % h_kv != 0) return -3;
+    if (n_rows <= 0 || (!rows && n_rows != s_q)) return -4;
+    if (causal && s_q > s_k) return -6;
+    if (window_left < -1 || (window_left >= 0 && !causal)) return -8;
+    const int64_t nq = (int64_t)batch * s_q * h_q * d, nk = (int64_t)batch * s_k * h_kv * d;
+    double *Q = (double *)malloc((size_t)nq * sizeof(double));
+    double *K = (double *)malloc((size_t)nk * sizeof(double));
+    double *V = (double *)malloc((size_t)nk * sizeof(double));
+    if (!Q || !K || !V) { free(Q); free(K); free(V); return -7; }
+    for (int64_t t = 0; t < nq; ++t) Q[t] = q_scale * e4m3_to_double(q[t]);
+    for (int64_t t = 0; t < nk; ++t) {
+        K[t] = k_scale * e4m3_to_double(k[t]);
+        V[t] = v_scale * e4m3_to_double(v[t]);
+    }
+    return forward_on_doubles(Q, K, V, batch, h_q, h_kv, s_q, s_k, d, causal, window_left,
+                              scale, rows, n_rows, o, lse, p);
+}
+
+/* Shared tail of both forward entries: takes ownership of Q, K, V. */
+static int forward_on_doubles(double *Q, double *K, double *V, int batch, int h_q, int h_kv,
+                              int s_q, int s_k, int d, int causal, int window_left,
+                              double scale, const int32_t *rows, int n_rows, double *o,
+                              double *lse, double *p)
+{
+    if (rows) {
+        for (int64_t t = 0; t < (int64_t)batch * h_q * n_rows; ++t)
+            if (rows[t] < 0 || rows[t] >= s_q) { free(Q); free(K); free(V); return -5; }
+    }
     const int chunk = 32;
     const int n_chunks = (n_rows + chunk - 1) / chunk;
     const int64_t n_tasks = (int64_t)batch * h_q * n_chunks;

@@ -462,6 +462,50 @@ def pin_bwd_invariants(lib):
     assert np.max(np.abs(dv[:, 22, 1] - want_v)) < 1e-12, "causal last key"
 
 
+# ------------------------------------------------------------------ FP8 inputs
+def _fp8_case(seed, b=2, hq=4, hkv=2, s_q=19, s_k=23, d=16):
+    g = torch.Generator().manual_seed(seed)
+    q = torch.randn(b, s_q, hq, d, generator=g).to(torch.float8_e4m3fn)
+    k = torch.randn(b, s_k, hkv, d, generator=g).to(torch.float8_e4m3fn)
+    v = torch.randn(b, s_k, hkv, d, generator=g).to(torch.float8_e4m3fn)
+    return q, k, v
+
+
+def pin_e4m3_decode_all_codes(lib):
+    """The oracle's E4M3 decoding of all 256 codes equals torch's float8_e4m3fn
+    conversion (NaN codes included)."""
+    codes = torch.arange(256, dtype=torch.uint8)
+    want = codes.view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    got = np.array([float(lib.oracle_e4m3_to_double(c)) for c in range(256)])
+    assert np.array_equal(np.isnan(want), np.isnan(got)), "E4M3 NaN codes"
+    ok = ~np.isnan(want)
+    assert np.array_equal(want[ok], got[ok]), "E4M3 values"
+
+
+def pin_fp8_forward_is_the_forward_of_the_dequantized_inputs(lib):
+    """With power-of-two scales every dequantized input is exactly a BF16
+    value, so the FP8 forward must equal the (pinned) BF16 forward on those
+    values bit for bit; with other scales it must equal torch's float64
+    SDPA on the dequantized values."""
+    q, k, v = _fp8_case(51)
+    for (qs, ks, vs) in [(0.5, 2.0, 0.25), (1.0, 1.0, 1.0)]:
+        for causal in (False, True):
+            o8, l8 = oracle.attn_fwd_fp8(q, k, v, qs, ks, vs, causal, 0.3, lib=lib)
+            qb = bf16(q.to(torch.float64).numpy() * qs)
+            kb = bf16(k.to(torch.float64).numpy() * ks)
+            vb = bf16(v.to(torch.float64).numpy() * vs)
+            o, l, _ = run(lib, qb, kb, vb, causal, 0.3)
+            assert np.array_equal(o8, o) and np.array_equal(l8, l), "FP8 vs BF16 forward"
+    qs, ks, vs = 0.37, 1.9, 0.61
+    o8, l8 = oracle.attn_fwd_fp8(q, k, v, qs, ks, vs, True, 0.3, lib=lib)
+    qt = (q.to(torch.float64) * qs).permute(0, 2, 1, 3)
+    kt = (k.to(torch.float64) * ks).permute(0, 2, 1, 3).repeat_interleave(2, 1)
+    vt = (v.to(torch.float64) * vs).permute(0, 2, 1, 3).repeat_interleave(2, 1)
+    mask = torch.ones(19, 23, dtype=torch.bool).tril(4)
+    want = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask, scale=0.3)
+    assert np.max(np.abs(o8 - want.numpy())) < 1e-12, "FP8 forward vs torch SDPA"
+
+
 ALL_PINS = [
     pin_rows_sum_to_one, pin_identical_v_rows, pin_zero_query, pin_causal_row0,
     pin_causal_rectangular_is_square_suffix, pin_causal_single_query_sees_every_key,
@@ -471,6 +515,7 @@ ALL_PINS = [
     pin_torch_sdpa_f64, pin_golden_closed_forms, pin_row_subset,
     pin_varlen_matches_block_diagonal_sdpa, pin_varlen_sequences_are_independent,
     pin_bwd_torch_autograd_f64, pin_bwd_finite_differences, pin_bwd_invariants,
+    pin_e4m3_decode_all_codes, pin_fp8_forward_is_the_forward_of_the_dequantized_inputs,
 ]
 
 

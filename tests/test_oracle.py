@@ -125,6 +125,12 @@ MUTANTS = {
     "bwd_dq_with_v": ("acc += dSrow[j] * Kb[", "acc += dSrow[j] * Vb["),
     "bwd_mask_off_by_one": ("if (causal && j > i + off) Prow[j]", "if (causal && j >= i + off) Prow[j]"),
     "bwd_gqa_overwrites": ("dVb[(int64_t)j * ks + c] += acc_v;", "dVb[(int64_t)j * ks + c] = acc_v;"),
+    # FP8 inputs
+    "e4m3_bias_8": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 8.0, e - 8)"),
+    "e4m3_subnormal_scale": ("ldexp((double)m, -9)", "ldexp((double)m, -10)"),
+    "e4m3_mantissa_sixteenths": ("ldexp(1.0 + m / 8.0, e - 7)", "ldexp(1.0 + m / 16.0, e - 7)"),
+    "fp8_v_takes_k_scale": ("V[t] = v_scale * e4m3_to_double(v[t]);",
+                            "V[t] = k_scale * e4m3_to_double(v[t]);"),
     "bwd_D_from_first_key": ("for (int j = 0; j < s_k; ++j) Di += Prow[j] * dProw[j];",
                              "for (int j = 0; j < 1; ++j) Di += Prow[j] * dProw[j];"),
 }
