@@ -53,7 +53,7 @@ def parse_args():
                     help="skip the per-configuration timing block")
     ap.add_argument("--config-launches", type=int, default=20,
                     help="timed launches per (configuration, mask) in that block")
-    ap.add_argument("--only", choices=["configs", "split"],
+    ap.add_argument("--only", choices=["configs", "split", "bwd", "fp8"],
                     help="run only the per-configuration block or only the split-KV cases "
                          "(for profiling) and print them as one JSON line")
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -385,6 +385,8 @@ def run_ours(args, world, rank, local):
     if world == 1 and not args.no_configs:
         line["configs"] = run_configs(args, peaks)
         line["configs"]["split_kv"] = run_split_cases(args, peaks)
+        line["configs"]["backward"] = run_backward(args, peaks)
+        line["configs"]["fp8"] = run_fp8(args, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         tfl, secs, n, steps, cores = oracle_sample_rate(w, args.cpu_seconds)
         line["cpu_baseline"] = {
@@ -511,6 +513,112 @@ def run_split_cases(args, peaks):
     return out
 
 
+BWD_WORKLOADS = ["mha_b8_h16_s4096", "mha_b4_h16_s8192", "gqa_b8_h16_kv2_s2048"]
+
+
+def run_backward(args, peaks):
+    """attn_bwd (prep + dK/dV + dQ launches) on a few workloads, both masks,
+    each call timed alone after an L2 flush; TFLOPS count 2.5x the forward's
+    FLOPs (the five GEMM-sized products of the standard backward, although
+    this one recomputes Q K^T and dO V^T for dQ)."""
+    from scaled_dot_product_10_b200 import attn
+    peak = float(peaks["bf16_tflops"])
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    out = {}
+    for name in BWD_WORKLOADS:
+        w = WORKLOADS[name]
+        q, k, v = (t.cuda() for t in workload_qkv(w))
+        dout = torch.randn(q.shape, generator=torch.Generator("cuda").manual_seed(w.seed + 50),
+                           device="cuda").to(torch.bfloat16)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = torch.empty(attn.bwd_workspace_bytes(w.batch, w.h_q, w.seq), dtype=torch.uint8,
+                         device="cuda")
+        entry = {}
+        for causal in MODES:
+            o, lse = attn.attn_fwd(q, k, v, causal=causal, scale=w.scale)
+
+            def call():
+                attn.attn_bwd(q, k, v, o, lse, dout, causal=causal, scale=w.scale, dq=dq, dk=dk,
+                              dv=dv, workspace=ws)
+            for _ in range(3):
+                call()
+            ev = []
+            for _ in range(max(5, args.config_launches // 2)):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                call()
+                b.record(stream)
+                ev.append((a, b))
+            torch.cuda.synchronize()
+            ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+            tf = 2.5 * w.flops(causal) / (ms * 1e-3) / 1e12
+            entry["causal" if causal else "noncausal"] = {"ms_per_call": ms, "tflops": tf,
+                                                          "frac": tf / peak}
+        rc = attn.attn_status()
+        if rc != attn.ATTN_OK:
+            raise attn.AttnError(rc, f"kernel status after backward {name}")
+        out[name] = entry
+        del q, k, v, dout, dq, dk, dv, ws
+    del flush
+    torch.cuda.empty_cache()
+    return out
+
+
+FP8_WORKLOADS = ["mha_b8_h16_s4096", "mha_b1_h16_s32768_k3", "gqa_b8_h16_kv2_s2048"]
+
+
+def run_fp8(args, peaks):
+    """attn_fwd_fp8 on E4M3 versions of a few workloads (per-tensor scales),
+    both masks, each launch timed alone after an L2 flush.  The fraction is
+    of the FP8 dense peak, taken as the measured BF16 peak x 2 (the nominal
+    FP8 / BF16 tensor-core ratio)."""
+    from scaled_dot_product_10_b200 import attn
+    from scaled_dot_product_10_b200.workloads import make_qkv_fp8
+    peak8 = 2.0 * float(peaks["bf16_tflops"])
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    out = {}
+    for name in FP8_WORKLOADS:
+        w = WORKLOADS[name]
+        q8, k8, v8, qs, ks, vs = make_qkv_fp8(w.batch, w.h_q, w.h_kv, w.seq, w.seq, seed=w.seed,
+                                              k_scale=w.k_scale)
+        q8, k8, v8 = q8.cuda(), k8.cuda(), v8.cuda()
+        o = torch.empty(q8.shape, dtype=torch.bfloat16, device="cuda")
+        lse = torch.empty((w.batch, w.h_q, w.seq), dtype=torch.float32, device="cuda")
+        entry = {}
+        for causal in MODES:
+            def call():
+                attn.attn_fwd_fp8(q8, k8, v8, qs, ks, vs, causal=causal, scale=w.scale, o=o,
+                                  lse=lse)
+            for _ in range(3):
+                call()
+            ev = []
+            for _ in range(args.config_launches):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                call()
+                b.record(stream)
+                ev.append((a, b))
+            torch.cuda.synchronize()
+            ms = statistics.median(a.elapsed_time(b) for a, b in ev)
+            tf = w.flops(causal) / (ms * 1e-3) / 1e12
+            entry["causal" if causal else "noncausal"] = {"ms_per_launch": ms, "tflops": tf,
+                                                          "frac_of_fp8_peak": tf / peak8}
+        rc = attn.attn_status()
+        if rc != attn.ATTN_OK:
+            raise attn.AttnError(rc, f"kernel status after FP8 {name}")
+        out[name] = entry
+        del q8, k8, v8, o, lse
+    del flush
+    torch.cuda.empty_cache()
+    return {"fp8_peak_tflops": peak8, "workloads": out}
+
+
 def run_e2e(args, w, q, k, v, world):
     """Same metric through the host-buffer C entry point: pinned host inputs,
     H2D copies, the forward, and D2H of O and LSE inside the timed region."""
@@ -557,7 +665,8 @@ def main():
         from scaled_dot_product_10_b200 import attn
         attn.load_library()
         peaks, _ = load_peaks()
-        part = run_configs(args, peaks) if args.only == "configs" else run_split_cases(args, peaks)
+        part = {"configs": run_configs, "split": run_split_cases,
+                "bwd": run_backward, "fp8": run_fp8}[args.only](args, peaks)
         print(json.dumps({"only": args.only, args.only: part}), flush=True)
         return 0
     try:

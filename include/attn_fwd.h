@@ -132,6 +132,29 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
                     void* stream);
 
 /*
+ * attn_fwd_fp8 -- the forward on FP8 E4M3 inputs with per-tensor scales
+ * (the FP8-GEMM / FP32-softmax precision split of the bjdmk.com.cn survey
+ * page, section 3, and the rkmt.cn page, section 3.1.1): the inputs stand for
+ * Q = q_scale * q, K = k_scale * k, V = v_scale * v, and the result is
+ * attn_fwd's on those values:
+ *
+ *   q, k, v   device, E4M3 bytes ("e4m3fn": no infinities) in attn_fwd's
+ *             layouts, one byte per element, 16-byte aligned
+ *   o, lse    as attn_fwd (BF16 O, FP32 natural-log LSE)
+ *   q_scale, k_scale, v_scale  finite per-tensor scales (ATTN_ERR_INVALID
+ *             otherwise)
+ *
+ * Q K^T and P V run on the tensor core in FP8 (kind::f8f6f4) with FP32
+ * accumulation; the softmax is FP32; the weights P are rounded to E4M3
+ * (stored as 2^6 P so the bulk of a row stays in E4M3's normal range).
+ * Arguments and errors otherwise as attn_fwd.  One launch; asynchronous;
+ * allocates nothing.
+ */
+int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal,
+                 float scale, float q_scale, float k_scale, float v_scale, void* stream);
+
+/*
  * attn_fwd_host -- the same forward on HOST buffers: copies q, k, v to the
  * device (cudaMemcpyAsync on `stream`), runs attn_fwd, copies o and lse back,
  * and returns without synchronising (the caller synchronises `stream` before

@@ -34,6 +34,8 @@ _SIGNATURES = [
     ("attn_bwd_workspace_bytes", ctypes.c_size_t, [_I, _I, _I]),
     ("attn_bwd", _I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, _I,
                       ctypes.c_float, _P, ctypes.c_size_t, _P]),
+    ("attn_fwd_fp8", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
+                          ctypes.c_float, ctypes.c_float, ctypes.c_float, _P]),
     ("attn_fwd_host", _I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _I, _I, ctypes.c_float,
                            _P, ctypes.c_size_t, _P]),
     ("attn_fwd_host_workspace_bytes", ctypes.c_size_t, [_I, _I, _I, _I, _I, _I]),
@@ -275,6 +277,31 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_bwd")
     return dq, dk, dv
+
+
+def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, causal: bool = False,
+                 scale: float | None = None, o=None, lse=None, stream=None):
+    """Forward on FP8 E4M3 CUDA tensors (torch.float8_e4m3fn) [batch, seq,
+    heads, 128] standing for q_scale * q, k_scale * k, v_scale * v.  Returns
+    (o BF16 [b, s_q, h_q, 128], lse FP32 [b, h_q, s_q])."""
+    import torch
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.dtype != torch.float8_e4m3fn or t.dim() != 4 or not t.is_contiguous() or not t.is_cuda:
+            raise ValueError(f"{name} must be a contiguous CUDA float8_e4m3fn [b, s, h, d]")
+    b, s_q, h_q, d = q.shape
+    bk, s_k, h_kv, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or bk != b or dk != d:
+        raise ValueError("q, k, v shapes disagree")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
+    rc = load_library().attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                     lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
+                                     int(bool(causal)), float(scale), float(q_scale),
+                                     float(k_scale), float(v_scale), _stream_handle(stream))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_fwd_fp8")
+    return o, lse
 
 
 def num_splits(b, h_q, h_kv, s_q, s_k, causal=False, d=128) -> int:

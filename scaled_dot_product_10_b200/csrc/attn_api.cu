@@ -66,6 +66,8 @@ int init_device(int dev, DeviceState** out) {
                 cudaSuccess ||
             cudaFuncSetAttribute(attn_fwd_sm100_kernel<true, true>, smem, Layout::kAlloc) !=
                 cudaSuccess ||
+            cudaFuncSetAttribute(attn_fwd_sm100_kernel<false, false, true>, smem,
+                                 SmemLayoutT<true>::kAlloc) != cudaSuccess ||
             cudaFuncSetAttribute(bwd::dq::attn_bwd_dq_kernel, smem, bwd::dq::Smem::kAlloc) !=
                 cudaSuccess ||
             cudaFuncSetAttribute(bwd::dkdv::attn_bwd_dkdv_kernel, smem,
@@ -94,6 +96,24 @@ bool encode_map(CUtensorMap* m, const void* base, int heads, int seq, int batch,
     cuuint32_t box[4] = {64, 1, box_rows, 1};
     cuuint32_t estr[4] = {1, 1, 1, 1};
     CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims,
+                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// [batch, seq, heads, 128] FP8 (one byte per element) as a 4-D tensor map,
+// box {128, 1, 128, 1}: a 128-row tile whose 128-byte rows are one swizzle
+// atom each.
+bool encode_map_fp8(CUtensorMap* m, const void* base, int heads, int seq, int batch) {
+    cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(heads),
+                          static_cast<cuuint64_t>(seq), static_cast<cuuint64_t>(batch)};
+    cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHeadDim),
+                             static_cast<cuuint64_t>(heads) * kHeadDim,
+                             static_cast<cuuint64_t>(seq) * heads * kHeadDim};
+    cuuint32_t box[4] = {128, 1, 128, 1};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), dims,
                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
@@ -157,7 +177,8 @@ struct Varlen {
 int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int batch,
                int h_q, int h_kv, int s_q, int s_k, int causal, int causal_offset, float scale,
                int n_splits, int kb_per_split, float* o_part, float* lse_part, void* stream,
-               int window_left = -1, const Varlen* varlen = nullptr) {
+               int window_left = -1, const Varlen* varlen = nullptr,
+               const float* fp8_scales = nullptr) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
     DeviceState* st = nullptr;
@@ -174,9 +195,16 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
         s_k = varlen->max_s_k;
     }
     CUtensorMap tq, tk, tv, to;
-    if (!encode_map(&tq, q, h_q, map_sq, map_b) || !encode_map(&tk, k, h_kv, map_sk, map_b) ||
-        !encode_map(&tv, v, h_kv, map_sk, map_b))
+    if (fp8_scales) {
+        if (!encode_map_fp8(&tq, q, h_q, map_sq, map_b) ||
+            !encode_map_fp8(&tk, k, h_kv, map_sk, map_b) ||
+            !encode_map_fp8(&tv, v, h_kv, map_sk, map_b))
+            return ATTN_ERR_CUDA;
+    } else if (!encode_map(&tq, q, h_q, map_sq, map_b) ||
+               !encode_map(&tk, k, h_kv, map_sk, map_b) ||
+               !encode_map(&tv, v, h_kv, map_sk, map_b)) {
         return ATTN_ERR_CUDA;
+    }
     // O is stored through a tensor map of the same shape as Q's (unused when
     // the launch writes FP32 partials instead).
     if (o != nullptr) {
@@ -220,10 +248,16 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     p.div_group = FastDiv::make(static_cast<uint32_t>(p.group));
     p.div_h_kv = FastDiv::make(static_cast<uint32_t>(h_kv));
     // The kernel exponentiates 2^((s - m) c) with c > 0: a negative scale
-    // negates the scores on the tensor core instead (see FwdParams).
-    const double c = std::fabs(static_cast<double>(scale)) * 1.4426950408889634;
+    // negates the scores on the tensor core instead (see FwdParams).  FP8
+    // inputs fold the Q and K scales into c and the V scale into 1 / l.
+    double eff = static_cast<double>(scale);
+    if (fp8_scales) eff *= static_cast<double>(fp8_scales[0]) * fp8_scales[1];
+    const double c = std::fabs(eff) * 1.4426950408889634;
     p.scale_log2 = static_cast<float>(c < 1e-30 ? 1e-30 : c);
-    p.idesc_qk = idesc_bf16_f32(kBlockM, kBlockN, 0, 0) | (scale < 0.f ? kIdescNegateA : 0u);
+    p.idesc_qk = (fp8_scales ? idesc_e4m3_f32(kBlockM, kBlockN, 0, 0)
+                             : idesc_bf16_f32(kBlockM, kBlockN, 0, 0)) |
+                 (eff < 0.0 ? kIdescNegateA : 0u);
+    p.v_scale = fp8_scales ? fp8_scales[2] : 1.f;
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
     p.o_part = o_part;
@@ -241,7 +275,10 @@ int launch_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
     const int grid = p.num_tiles < st->num_sms ? p.num_tiles : st->num_sms;
     const cudaStream_t cs = static_cast<cudaStream_t>(stream);
     const bool win = window_left >= 0;
-    if (!varlen && !win)
+    if (fp8_scales)
+        attn_fwd_sm100_kernel<false, false, true>
+            <<<grid, kThreads, SmemLayoutT<true>::kAlloc, cs>>>(tq, tk, tv, to, p);
+    else if (!varlen && !win)
         attn_fwd_sm100_kernel<false, false><<<grid, kThreads, Layout::kAlloc, cs>>>(tq, tk, tv, to, p);
     else if (!varlen)
         attn_fwd_sm100_kernel<true, false><<<grid, kThreads, Layout::kAlloc, cs>>>(tq, tk, tv, to, p);
@@ -408,8 +445,16 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
         !encode_map(&tdk, dk, h_kv, s_k, batch) || !encode_map(&tdv, dv, h_kv, s_k, batch))
         return ATTN_ERR_CUDA;
 
+    // Sections of 4 heads keep the streamed tiles of the heads in flight in
+    // L2; launches with few items (at most 4 rounds of SMs) use one section
+    // so their longest-first order can balance the CTAs.
+    constexpr int kHeadsPerSection = 4;
+    const int rounds4 = 4 * st->num_sms;
+
     // 2. dK, dV: one item per (key block, batch, key/value head).
     p.num_items = batch * h_kv * p.n_kb;
+    p.section = p.num_items <= rounds4 ? batch * h_kv : kHeadsPerSection;
+    if (p.section > batch * h_kv) p.section = batch * h_kv;
     int grid = p.num_items < st->num_sms ? p.num_items : st->num_sms;
     bwd::dkdv::attn_bwd_dkdv_kernel<<<grid, bwd::kThreads, bwd::dkdv::Smem::kAlloc, cs>>>(
         tq64, tk, tv, tdo64, tdk, tdv, p);
@@ -417,12 +462,28 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
 
     // 3. dQ: one item per (query block, batch, query head).
     p.num_items = batch * h_q * p.n_qb;
+    p.section = p.num_items <= rounds4 ? batch * h_q : kHeadsPerSection;
+    if (p.section > batch * h_q) p.section = batch * h_q;
     grid = p.num_items < st->num_sms ? p.num_items : st->num_sms;
     bwd::dq::attn_bwd_dq_kernel<<<grid, bwd::kThreads, bwd::dq::Smem::kAlloc, cs>>>(tq, tk, tv,
                                                                                      tdo, tdq, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     g_last_launches = 3;
     return ATTN_OK;
+}
+
+extern "C" int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal,
+                            float scale, float q_scale, float k_scale, float v_scale,
+                            void* stream) {
+    const int rc = validate(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale);
+    if (rc != ATTN_OK) return rc;
+    if (!std::isfinite(q_scale) || !std::isfinite(k_scale) || !std::isfinite(v_scale))
+        return ATTN_ERR_INVALID;
+    const float scales[3] = {q_scale, k_scale, v_scale};
+    const int n_kb = (s_k + kBlockN - 1) / kBlockN;
+    return launch_fwd(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, causal, s_k - s_q, scale, 1,
+                      n_kb, nullptr, nullptr, stream, -1, nullptr, scales);
 }
 
 extern "C" int attn_fwd_num_splits(int batch, int h_q, int h_kv, int s_q, int s_k, int d,

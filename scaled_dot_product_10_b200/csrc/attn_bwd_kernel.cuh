@@ -53,6 +53,12 @@ struct BwdParams {
     int causal_offset;     // s_k - s_q
     int window_left;       // -1: none
     int num_items;
+    // Items are grouped in sections of `section` heads ((batch, query head)
+    // for dQ, (batch, key/value head) for dK/dV): inside a section the order
+    // is longest first, then head, so the CTAs running at one time share the
+    // few heads whose streamed tiles stay in L2.  section = all heads when
+    // the launch has too few items to balance per section.
+    int section;
     FastDiv div_n_qb;      // n_qb
     FastDiv div_n_kb;      // n_kb
     FastDiv div_h_q;       // h_q
@@ -140,16 +146,21 @@ struct Smem {
 };
 constexpr int kStages = 2;
 
-// Item t -> (batch, query head, query block), longest causal work first:
-// query block descending, then (batch, head).
+// Item t -> (batch, query head, query block): by section of heads, then
+// query block descending (longest causal work first), then head.
 struct Cursor {
     int round, t;
     int b, h, g, qb, n;  // n: key blocks visited
     int kb_lo;           // first key block (sliding window)
     __device__ __forceinline__ void decode(const BwdParams& p) {
+        // Once per item: plain divisions are fine.
         const int bh_count = p.batch * p.h_q;
-        const int rank = t / bh_count;  // once per item: plain division is fine
-        const int bh = t - rank * bh_count;
+        const int per_sec = p.section * p.n_qb;
+        const int sec = t / per_sec;
+        const int in_sec = min(p.section, bh_count - sec * p.section);  // heads in this section
+        const int r = t - sec * per_sec;
+        const int rank = r / in_sec;
+        const int bh = sec * p.section + (r - rank * in_sec);
         qb = p.n_qb - 1 - rank;
         b = p.div_h_q.div(bh);
         h = bh - b * p.h_q;
@@ -526,9 +537,9 @@ struct Smem {
     static constexpr int kAlloc = kBytes + 1024;
 };
 
-// Item t -> (key block, batch, key/value head): key block ascending (under
-// the causal mask the first key blocks are seen by the most query rows:
-// longest first), then (batch, head).  The item walks the query heads of
+// Item t -> (key block, batch, key/value head): by section of heads, then
+// key block ascending (under the causal mask the first key blocks are seen
+// by the most query rows: longest first), then head.  The item walks the query heads of
 // the group and, for each, the 64-row query blocks that see the key block.
 struct Cursor {
     int round, t;
@@ -536,8 +547,12 @@ struct Cursor {
     int qlo, nq;  // query blocks qlo .. qlo + nq - 1 per head
     __device__ __forceinline__ void decode(const BwdParams& p) {
         const int bg_count = p.batch * p.h_kv;
-        kb = t / bg_count;
-        const int bg = t - kb * bg_count;
+        const int per_sec = p.section * p.n_kb;
+        const int sec = t / per_sec;
+        const int in_sec = min(p.section, bg_count - sec * p.section);
+        const int r = t - sec * per_sec;
+        kb = r / in_sec;
+        const int bg = sec * p.section + (r - kb * in_sec);
         b = p.div_h_kv.div(bg);
         g = bg - b * p.h_kv;
         int lo = 0, hi = p.n_qb64;
@@ -587,7 +602,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
-    const float* sLD = reinterpret_cast<const float*>(smem + L::kLD);
+
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
@@ -797,8 +812,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (p.window_left >= 0)
                     hi = min(hi, key + p.window_left - p.causal_offset - qb * kBlockQ);
                 const uint32_t slot = gs & 1;
-                const float* sL = sLD + slot * 128;
-                const float* sD = sL + 64;
+                const uint32_t sL = sbase + L::kLD + slot * 512;  // L[64], then D[64]
+                const uint32_t sD = sL + 256;
                 float pt[64];
                 // L and D of this step's rows arrive with its Q / dO tiles
                 // (the slot is refilled only after this step's dK MMA, which
@@ -818,9 +833,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bar(L::bSFree));
 #pragma unroll
-                for (int k = 0; k < 64; ++k) {
-                    const float x = ptx::ex2(fmaf(pt[k], c2, -sL[k]));
-                    pt[k] = (k >= lo && k <= hi) ? x : 0.f;
+                for (int k4 = 0; k4 < 16; ++k4) {
+                    const float4 l4 = ptx::ld_shared_f4(sL + 16 * k4);  // same address: broadcast
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int k = 4 * k4 + e;
+                        const float x = ptx::ex2(fmaf(pt[k], c2, -lv[e]));
+                        pt[k] = (k >= lo && k <= hi) ? x : 0.f;
+                    }
                 }
                 // P^T -> BF16 into its tile once the last dV MMA has read it.
                 if (gs > 0 && !wait_bar_warp(bar(L::bPTFree), (gs - 1) & 1, wc)) return;
@@ -844,8 +865,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::tmem_ld32(dp_tm + q * 32, dr);
                     ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 32; ++k)
-                        pt[q * 32 + k] = pt[q * 32 + k] * (__uint_as_float(dr[k]) - sD[q * 32 + k]);
+                    for (int k4 = 0; k4 < 8; ++k4) {
+                        const float4 d4 = ptx::ld_shared_f4(sD + 4 * (q * 32 + 4 * k4));
+                        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            const int k = 4 * k4 + e;
+                            pt[q * 32 + k] = pt[q * 32 + k] * (__uint_as_float(dr[k]) - dv4[e]);
+                        }
+                    }
                 }
                 ptx::tc_fence_before();
                 __syncwarp();

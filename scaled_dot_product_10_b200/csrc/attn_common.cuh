@@ -91,6 +91,7 @@ struct FwdParams {
     const int* cu_q;
     const int* cu_k;
     int total_q;
+    float v_scale;  // FP8 kernel only: V = v_scale * E4M3 values (1 otherwise)
 };
 
 // ------------------------------------------------------------------ waits

@@ -203,14 +203,20 @@ struct PairCursor {
 };
 
 // ------------------------------------------------------------------ layout
-constexpr int kKStages = 1;  // K tiles in flight
-constexpr int kVStages = 2;  // V tiles in flight
-struct SmemLayout {
+// BF16: 32 KiB Q/K/V/P tiles, a K ring of 1 and a V ring of 2, O staged in
+// the block's P tile.  FP8 (E4M3): 16 KiB tiles (a 128-byte row is one
+// swizzle atom), deeper rings, and a BF16 O staging tile per block.
+template <bool kFp8>
+struct SmemLayoutT {
+    static constexpr int kTile = kFp8 ? kTileBytes / 2 : kTileBytes;
+    static constexpr int kKStages = kFp8 ? 2 : 1;  // K tiles in flight
+    static constexpr int kVStages = kFp8 ? 3 : 2;  // V tiles in flight
     static constexpr int kQ = 0;                              // Q0, Q1
-    static constexpr int kP = 2 * kTileBytes;                 // P0, P1
-    static constexpr int kK = 4 * kTileBytes;                 // K ring
-    static constexpr int kV = kK + kKStages * kTileBytes;     // V ring
-    static constexpr int kBars = kV + kVStages * kTileBytes;  // mbarriers
+    static constexpr int kP = 2 * kTile;                      // P0, P1
+    static constexpr int kK = 4 * kTile;                      // K ring
+    static constexpr int kV = kK + kKStages * kTile;          // V ring
+    static constexpr int kO = kV + kVStages * kTile;          // FP8: O staging (2 x 32 KiB)
+    static constexpr int kBars = kO + (kFp8 ? 2 * kTileBytes : 0);  // mbarriers
     static constexpr int bQFull = 0, bQEmpty = 2, bKFull = 4, bKEmpty = 4 + kKStages,
                          bVFull = 4 + 2 * kKStages, bVEmpty = bVFull + kVStages,
                          bSFull = bVEmpty + kVStages,
@@ -219,10 +225,21 @@ struct SmemLayout {
                          bOStaged = bDrain + 2, bOStored = bOStaged + 2,
                          kNumBars = bOStored + 2;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
+    // Leading offset of the V descriptor (MN-major): the second 64-column
+    // head-dim half for BF16; FP8 rows are one atom wide, so it is not used.
+    static constexpr uint32_t kFp8Lbo = kFp8 ? kTile : kHalfTileBytes;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
     static constexpr int kAlloc = kBytes + 1024;  // slack for 1024-byte alignment
 };
+using SmemLayout = SmemLayoutT<false>;
+
+// FP8 P: the lazy rescale threshold is 2^2 and the weights are stored as
+// 2^6 * P, so a row's weights span up to 2^8 at the top and keep E4M3's
+// normal range (down to 2^-6, i.e. P >= 2^-12) for the bulk of the mass;
+// the 2^6 cancels in O / l and is taken out of the LSE.
+constexpr float kFp8RescaleThresholdLog2 = 2.0f;
+constexpr float kFp8PBiasLog2 = 6.0f;
 
 // ------------------------------------------------------------------ exponentials
 // P = 2^(s c - m c) for one 128-key row on the MUFU ex2 unit: FP32 row sum
@@ -230,13 +247,16 @@ struct SmemLayout {
 // shared-memory P tile (16-byte chunk cc at row_base + (cc / 8) * 16 KiB +
 // ((cc % 8) ^ xor) * 16).  When `pass_turn` is set the warp arrives on the
 // turn barrier after kTurnChunk chunks.
+template <bool kFp8>
 __device__ __forceinline__ void exp_row(const float (&s)[128], uint64_t c2x2, uint64_t nmc2,
                                         uint32_t p_row, uint32_t p_xor, float& sum_a,
                                         float& sum_b, bool pass_turn, uint32_t turn, int lane) {
     uint64_t sum2a = ptx::f2_pack(0.f, 0.f), sum2b = sum2a;
+    uint32_t w8[4];  // FP8: two 8-key groups make one 16-byte chunk
 #pragma unroll
     for (int cc = 0; cc < 16; ++cc) {
         uint32_t w[4];
+        float pv[8];
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int e0 = 8 * cc + 2 * k;
@@ -247,10 +267,25 @@ __device__ __forceinline__ void exp_row(const float (&s)[128], uint64_t c2x2, ui
             const uint64_t e = ptx::f2_pack(p0, p1);
             if (k & 1) sum2b = ptx::f2_add(sum2b, e);
             else sum2a = ptx::f2_add(sum2a, e);
-            w[k] = ptx::pack_bf16x2(p0, p1);
+            if constexpr (kFp8) {
+                pv[2 * k] = p0;
+                pv[2 * k + 1] = p1;
+            } else {
+                w[k] = ptx::pack_bf16x2(p0, p1);
+            }
         }
-        ptx::st_shared_v4(p_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ p_xor) << 4), w[0],
-                          w[1], w[2], w[3]);
+        if constexpr (kFp8) {
+            // Row of 128 E4M3 weights = one 128-byte swizzle atom row:
+            // 16-byte chunk c (keys 16c .. 16c + 15) at ((c ^ xor) * 16).
+            w8[2 * (cc & 1)] = ptx::pack_e4m3x4(pv[0], pv[1], pv[2], pv[3]);
+            w8[2 * (cc & 1) + 1] = ptx::pack_e4m3x4(pv[4], pv[5], pv[6], pv[7]);
+            if (cc & 1)
+                ptx::st_shared_v4(p_row + ((((cc >> 1) & 7) ^ p_xor) << 4), w8[0], w8[1], w8[2],
+                                  w8[3]);
+        } else {
+            ptx::st_shared_v4(p_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ p_xor) << 4),
+                              w[0], w[1], w[2], w[3]);
+        }
         if (cc == kTurnChunk - 1 && pass_turn) {
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(turn);
@@ -265,11 +300,12 @@ __device__ __forceinline__ void exp_row(const float (&s)[128], uint64_t c2x2, ui
 
 // ------------------------------------------------------------------ softmax
 // One softmax warpgroup: thread r owns query row r of its block (TMEM lane r).
-template <bool kWindow, bool kVarlen>
+template <bool kWindow, bool kVarlen, bool kFp8>
 __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorMap* tm_o,
                                              const WaitCtx& wc, uint32_t tmem, uint32_t sP,
-                                             uint32_t bars, int wg, int warp_in_wg, int lane) {
-    using L = SmemLayout;
+                                             uint32_t sO, uint32_t bars, int wg, int warp_in_wg,
+                                             int lane) {
+    using L = SmemLayoutT<kFp8>;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
     const int r = warp_in_wg * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(warp_in_wg * 32) << 16;
@@ -282,8 +318,13 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
     // This row of P in shared memory (K-major, 128-byte swizzle, two 64-key
     // halves 16 KiB apart): 16-byte chunk c of the row lands at
     // row_base + (c / 8) * 16 KiB + ((c % 8) ^ (r % 8)) * 16.
-    const uint32_t p_row = sP + wg * kTileBytes + (r >> 3) * 1024 + (r & 7) * 128;
+    const uint32_t p_row = sP + wg * L::kTile + (r >> 3) * 1024 + (r & 7) * 128;
     const uint32_t p_xor = static_cast<uint32_t>(r & 7);
+    // The BF16 O tile of this block is staged at o_tile before its TMA store
+    // (the block's P tile for BF16 inputs).
+    const uint32_t o_tile = (kFp8 ? sO : sP) + wg * kTileBytes;
+    const uint32_t o_row = o_tile + (r >> 3) * 1024 + (r & 7) * 128;
+    constexpr float kThreshold = kFp8 ? kFp8RescaleThresholdLog2 : kRescaleThresholdLog2;
     const float c2 = p.scale_log2;
     const uint64_t c2x2 = ptx::f2_pack(c2, c2);
 
@@ -381,13 +422,14 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
             bool rescale = false;
             if (m_run == -CUDART_INF_F) {
                 m_run = mx;
-            } else if ((mx - m_run) * c2 > kRescaleThresholdLog2) {
+            } else if ((mx - m_run) * c2 > kThreshold) {
                 alpha = ptx::ex2((m_run - mx) * c2);
                 m_run = mx;
                 rescale = true;
             }
             const float m_ref = (m_run == -CUDART_INF_F) ? 0.f : m_run;
-            const float neg_mc = -m_ref * c2;
+            float neg_mc = -m_ref * c2;
+            if constexpr (kFp8) neg_mc += kFp8PBiasLog2;  // weights stored as 2^6 P
 
             // The previous P V of this block must be done before its P
             // buffer is rewritten (and before O is rescaled).
@@ -430,8 +472,8 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
             }
             if (turn && m > 0 && !wait_bar_warp(b_turn, (m - 1) & 1, wc)) return;
             float sum_a = 0.f, sum_b = 0.f;
-            exp_row(s, c2x2, ptx::f2_pack(neg_mc, neg_mc), p_row, p_xor, sum_a, sum_b, turn, b_turn,
-                    lane);
+            exp_row<kFp8>(s, c2x2, ptx::f2_pack(neg_mc, neg_mc), p_row, p_xor, sum_a, sum_b, turn,
+                          b_turn, lane);
             // Make P visible to the tensor core (async proxy) and hand it over.
             ptx::fence_proxy_async_smem();
             __syncwarp();
@@ -449,8 +491,11 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
                     // queries may see no key: O = 0 (LSE = -inf).
                     inv_l = l_run > 0.f ? inv_l : 0.f;
                 }
+                if constexpr (kFp8) inv_l *= p.v_scale;  // V = v_scale * E4M3 values
                 const uint64_t il2 = ptx::f2_pack(inv_l, inv_l);
-                const float lse_row = (m_ref * c2 + __log2f(l_run)) * 0.69314718055994531f;
+                float log2_l = __log2f(l_run);
+                if constexpr (kFp8) log2_l -= kFp8PBiasLog2;
+                const float lse_row = (m_ref * c2 + log2_l) * 0.69314718055994531f;
                 const size_t row_id = (static_cast<size_t>(c.b) * p.h_q + c.h) * p.s_q + row;
                 if (p.o_part != nullptr) {
                     // A row of a key shard may see none of its keys (l = 0):
@@ -523,7 +568,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
                             for (int k = 0; k < 4; ++k) {
                                 const int cc = 4 * q + k;
                                 ptx::st_shared_v4(
-                                    p_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ p_xor) << 4),
+                                    o_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ p_xor) << 4),
                                     w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
                             }
                         } else if (row_ok) {
@@ -544,7 +589,7 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
                     if (r == 0) {
                         if (!wait_bar(b_ostaged, stored & 1, wc)) return;
                         if (tma_tile) {
-                            const uint32_t tile = sP + wg * kTileBytes;
+                            const uint32_t tile = o_tile;
                             int row0 = qb * kBlockM, bc = c.b;
                             if constexpr (kVarlen) {
                                 row0 += c.q_row0;  // packed rows, batch extent 1
@@ -574,14 +619,14 @@ __device__ __forceinline__ void softmax_role(const FwdParams& p, const CUtensorM
 }
 
 // ------------------------------------------------------------------ kernel
-template <bool kWindow, bool kVarlen>
+template <bool kWindow, bool kVarlen, bool kFp8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     attn_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __grid_constant__ CUtensorMap tm_v,
                           const __grid_constant__ CUtensorMap tm_o,
                           const __grid_constant__ FwdParams p) {
-    using L = SmemLayout;
+    using L = SmemLayoutT<kFp8>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -590,6 +635,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t sP = sbase + L::kP;
     const uint32_t sK = sbase + L::kK;
     const uint32_t sV = sbase + L::kV;
+    const uint32_t sO = sbase + L::kO;
     const uint32_t bars = sbase + L::kBars;
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
@@ -610,11 +656,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(bar(L::bOStaged + i), 4);  // the 4 warps' rows are staged
             ptx::mbar_init(bar(L::bOStored + i), 1);  // TMA has read the staged tile
         }
-        for (int i = 0; i < kKStages; ++i) {
+        for (int i = 0; i < L::kKStages; ++i) {
             ptx::mbar_init(bar(L::bKFull + i), 1);
             ptx::mbar_init(bar(L::bKEmpty + i), 2);  // one arrival per MMA issuer
         }
-        for (int i = 0; i < kVStages; ++i) {
+        for (int i = 0; i < L::kVStages; ++i) {
             ptx::mbar_init(bar(L::bVFull + i), 1);
             ptx::mbar_init(bar(L::bVEmpty + i), 2);
         }
@@ -652,28 +698,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             auto load_tile = [&](const CUtensorMap* tm, uint32_t dst, uint32_t full,
                                  const PairCursor<kWindow, kVarlen>& c,
                                  int j) {
-                ptx::mbar_arrive_expect_tx(full, kTileBytes);
+                ptx::mbar_arrive_expect_tx(full, L::kTile);
                 int key0 = (c.kb0 + j) * kBlockN, bc = c.b;
                 if constexpr (kVarlen) {
                     key0 += c.k_row0;  // packed keys, batch extent 1
                     bc = 0;
                 }
                 ptx::tma_load_4d(dst, tm, full, 0, c.g, key0, bc, pol_kv);
-                ptx::tma_load_4d(dst + kHalfTileBytes, tm, full, 64, c.g, key0, bc, pol_kv);
+                if constexpr (!kFp8)
+                    ptx::tma_load_4d(dst + kHalfTileBytes, tm, full, 64, c.g, key0, bc, pol_kv);
             };
             auto load_k = [&](const PairCursor<kWindow, kVarlen>& c, int j) -> bool {
-                const int slot = k_loads % kKStages;
-                if (!wait_bar(bar(L::bKEmpty + slot), ((k_loads / kKStages) & 1) ^ 1, wc))
+                const int slot = k_loads % L::kKStages;
+                if (!wait_bar(bar(L::bKEmpty + slot), ((k_loads / L::kKStages) & 1) ^ 1, wc))
                     return false;
-                load_tile(&tm_k, sK + slot * kTileBytes, bar(L::bKFull + slot), c, j);
+                load_tile(&tm_k, sK + slot * L::kTile, bar(L::bKFull + slot), c, j);
                 ++k_loads;
                 return true;
             };
             auto load_v = [&](const PairCursor<kWindow, kVarlen>& c, int j) -> bool {
-                const int slot = v_loads % kVStages;
-                if (!wait_bar(bar(L::bVEmpty + slot), ((v_loads / kVStages) & 1) ^ 1, wc))
+                const int slot = v_loads % L::kVStages;
+                if (!wait_bar(bar(L::bVEmpty + slot), ((v_loads / L::kVStages) & 1) ^ 1, wc))
                     return false;
-                load_tile(&tm_v, sV + slot * kTileBytes, bar(L::bVFull + slot), c, j);
+                load_tile(&tm_v, sV + slot * L::kTile, bar(L::bVFull + slot), c, j);
                 ++v_loads;
                 return true;
             };
@@ -687,16 +734,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                         ok = false;
                         continue;
                     }
-                    const uint32_t dst = sQ + i * kTileBytes;
+                    const uint32_t dst = sQ + i * L::kTile;
                     int row0 = (c.qb0 + i) * kBlockM, bc = c.b;
                     if constexpr (kVarlen) {
                         row0 += c.q_row0;
                         bc = 0;
                     }
-                    ptx::mbar_arrive_expect_tx(bar(L::bQFull + i), kTileBytes);
+                    ptx::mbar_arrive_expect_tx(bar(L::bQFull + i), L::kTile);
                     ptx::tma_load_4d(dst, &tm_q, bar(L::bQFull + i), 0, c.h, row0, bc, pol_q);
-                    ptx::tma_load_4d(dst + kHalfTileBytes, &tm_q, bar(L::bQFull + i), 64, c.h,
-                                     row0, bc, pol_q);
+                    if constexpr (!kFp8)
+                        ptx::tma_load_4d(dst + kHalfTileBytes, &tm_q, bar(L::bQFull + i), 64, c.h,
+                                         row0, bc, pol_q);
                     ++q_loads[i];
                 }
                 // Issue order = the MMA warp's consumption order:
@@ -709,13 +757,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             // Drain: every issued copy must land before the CTA may exit.
-            for (int i = 0; i < kKStages && i < static_cast<int>(k_loads); ++i) {
+            for (int i = 0; i < L::kKStages && i < static_cast<int>(k_loads); ++i) {
                 const uint32_t f = k_loads - 1 - i;
-                wait_slow(bar(L::bKFull + f % kKStages), (f / kKStages) & 1, wc, false);
+                wait_slow(bar(L::bKFull + f % L::kKStages), (f / L::kKStages) & 1, wc, false);
             }
-            for (int i = 0; i < kVStages && i < static_cast<int>(v_loads); ++i) {
+            for (int i = 0; i < L::kVStages && i < static_cast<int>(v_loads); ++i) {
                 const uint32_t f = v_loads - 1 - i;
-                wait_slow(bar(L::bVFull + f % kVStages), (f / kVStages) & 1, wc, false);
+                wait_slow(bar(L::bVFull + f % L::kVStages), (f / L::kVStages) & 1, wc, false);
             }
 #pragma unroll
             for (int i = 0; i < 2; ++i)
@@ -735,28 +783,30 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t s_cnt = 0, pv_cnt = 0;   // Q K^T / P V groups issued
             bool ok = true;
             // Descriptor low words (start address >> 4 | leading offset).
-            const uint32_t q_lo = desc_lo_sw128(sQ + i * kTileBytes, 16);
-            const uint32_t p_lo = desc_lo_sw128(sP + i * kTileBytes, 16);
+            const uint32_t q_lo = desc_lo_sw128(sQ + i * L::kTile, 16);
+            const uint32_t p_lo = desc_lo_sw128(sP + i * L::kTile, 16);
             const uint32_t k_lo = desc_lo_sw128(sK, 16);
-            const uint32_t v_lo = desc_lo_sw128(sV, kHalfTileBytes);
+            const uint32_t v_lo = desc_lo_sw128(sV, L::kFp8Lbo);
             const uint32_t s_tm = tmem + i * 128, o_tm = tmem + 256 + i * 128;
             auto wait_k = [&]() -> bool {
-                return wait_bar(bar(L::bKFull + k_used % kKStages), (k_used / kKStages) & 1, wc);
+                return wait_bar(bar(L::bKFull + k_used % L::kKStages), (k_used / L::kKStages) & 1,
+                                wc);
             };
             auto wait_v = [&]() -> bool {
-                return wait_bar(bar(L::bVFull + v_used % kVStages), (v_used / kVStages) & 1, wc);
+                return wait_bar(bar(L::bVFull + v_used % L::kVStages), (v_used / L::kVStages) & 1,
+                                wc);
             };
             // A tile this block does not use: once it has landed (so the slot's
             // previous use is released), give up this issuer's share of it.
             auto skip_k = [&]() -> bool {
                 if (!wait_k()) return false;
-                ptx::mbar_arrive(bar(L::bKEmpty + k_used % kKStages));
+                ptx::mbar_arrive(bar(L::bKEmpty + k_used % L::kKStages));
                 ++k_used;
                 return true;
             };
             auto skip_v = [&]() -> bool {
                 if (!wait_v()) return false;
-                ptx::mbar_arrive(bar(L::bVEmpty + v_used % kVStages));
+                ptx::mbar_arrive(bar(L::bVEmpty + v_used % L::kVStages));
                 ++v_used;
                 return true;
             };
@@ -765,18 +815,27 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_k()) return false;
                 if (s_cnt > 0 && !wait_bar(bar(L::bSFree + i), (s_cnt - 1) & 1, wc)) return false;
                 ptx::tc_fence_after();
-                const uint32_t ka = k_lo + (((k_used % kKStages) * kTileBytes) >> 4);
+                const uint32_t ka = k_lo + (((k_used % L::kKStages) * L::kTile) >> 4);
+                if constexpr (kFp8) {
+                    // K-major, 128-byte swizzle: 32 E4M3 (32 bytes) per step;
+                    // a 128-element row is one swizzle atom.
 #pragma unroll
-                for (int k = 0; k < kHeadDim / 16; ++k) {
-                    // K-major, 128-byte swizzle: 16 BF16 (32 bytes) per step
-                    // inside a 64-column half; the second half is 16 KiB on.
-                    const uint32_t off = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
-                    ptx::mma_ss(s_tm, desc_from_lo(q_lo + off), desc_from_lo(ka + off), idesc_qk,
-                                k > 0 ? 1u : 0u);
+                    for (int k = 0; k < kHeadDim / 32; ++k)
+                        ptx::mma_ss_f8(s_tm, desc_from_lo(q_lo + 2 * k), desc_from_lo(ka + 2 * k),
+                                       idesc_qk, k > 0 ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < kHeadDim / 16; ++k) {
+                        // K-major, 128-byte swizzle: 16 BF16 (32 bytes) per step
+                        // inside a 64-column half; the second half is 16 KiB on.
+                        const uint32_t off = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
+                        ptx::mma_ss(s_tm, desc_from_lo(q_lo + off), desc_from_lo(ka + off),
+                                    idesc_qk, k > 0 ? 1u : 0u);
+                    }
                 }
                 ptx::mma_commit(bar(L::bSFull + i));
                 if (last_of_pair) ptx::mma_commit(bar(L::bQEmpty + i));
-                ptx::mma_commit(bar(L::bKEmpty + k_used % kKStages));
+                ptx::mma_commit(bar(L::bKEmpty + k_used % L::kKStages));
                 ++k_used;
                 ++s_cnt;
                 return true;
@@ -786,19 +845,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait_v()) return false;
                 if (!wait_bar(bar(L::bPFull + i), pv_cnt & 1, wc)) return false;
                 ptx::tc_fence_after();
-                const uint32_t va = v_lo + (((v_used % kVStages) * kTileBytes) >> 4);
+                const uint32_t va = v_lo + (((v_used % L::kVStages) * L::kTile) >> 4);
+                if constexpr (kFp8) {
+                    // A = P (E4M3, K-major like Q): 32 keys (32 bytes) per
+                    // step; B = V, MN-major (head dim contiguous, one
+                    // 128-byte atom wide): 32 keys = 32 rows = 4 KiB per step.
+                    constexpr uint32_t kIdescPV8 = idesc_e4m3_f32(kBlockM, kHeadDim, 0, 1);
 #pragma unroll
-                for (int k = 0; k < kBlockN / 16; ++k) {
-                    // A = P (K-major like Q); B = V, MN-major (head dim
-                    // contiguous): 16 keys = two 8-row swizzle atoms = 2 KiB
-                    // per step; the two 64-wide head-dim halves are 16 KiB apart.
-                    const uint32_t off = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
-                    ptx::mma_ss(o_tm, desc_from_lo(p_lo + off),
-                                desc_from_lo(va + ((k * 2048) >> 4)), kIdescPV,
-                                (acc || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < kBlockN / 32; ++k)
+                        ptx::mma_ss_f8(o_tm, desc_from_lo(p_lo + 2 * k),
+                                       desc_from_lo(va + ((k * 4096) >> 4)), kIdescPV8,
+                                       (acc || k > 0) ? 1u : 0u);
+                } else {
+#pragma unroll
+                    for (int k = 0; k < kBlockN / 16; ++k) {
+                        // A = P (K-major like Q); B = V, MN-major (head dim
+                        // contiguous): 16 keys = two 8-row swizzle atoms = 2 KiB
+                        // per step; the two 64-wide head-dim halves are 16 KiB apart.
+                        const uint32_t off = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
+                        ptx::mma_ss(o_tm, desc_from_lo(p_lo + off),
+                                    desc_from_lo(va + ((k * 2048) >> 4)), kIdescPV,
+                                    (acc || k > 0) ? 1u : 0u);
+                    }
                 }
                 ptx::mma_commit(bar(L::bOFull + i));
-                ptx::mma_commit(bar(L::bVEmpty + v_used % kVStages));
+                ptx::mma_commit(bar(L::bVEmpty + v_used % L::kVStages));
                 ++v_used;
                 ++pv_cnt;
                 return true;
@@ -866,7 +937,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp < 8) {
         ptx::reg_alloc<kRegsSoftmax>();
-        softmax_role<kWindow, kVarlen>(p, &tm_o, wc, tmem, sP, bars, warp >> 2, warp & 3, lane);
+        softmax_role<kWindow, kVarlen, kFp8>(p, &tm_o, wc, tmem, sP, sO, bars, warp >> 2, warp & 3,
+                                             lane);
     } else {
         ptx::reg_dealloc<kRegsControl>();  // idle warps of the control warpgroup
     }

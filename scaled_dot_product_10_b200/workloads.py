@@ -121,3 +121,23 @@ def sample_rows(batch: int, h_q: int, s_q: int, n: int, seed: int,
             extra = rng.choice(pool, size=n - len(fixed), replace=False)
             out[b, h] = np.sort(np.concatenate([np.array(fixed, dtype=np.int64), extra])).astype(np.int32)
     return out
+
+
+def make_qkv_fp8(batch: int, h_q: int, h_kv: int, s_q: int, s_k: int, seed: int,
+                 d: int = HEAD_DIM, k_scale: float = 1.0):
+    """FP8 E4M3 Q, K, V with per-tensor scales: the same N(0, 1) draws as
+    :func:`make_qkv` (FP32, before any rounding), each tensor divided by its
+    scale amax / 448 and rounded to E4M3 (torch's conversion).  Returns
+    (q8, k8, v8, q_scale, k_scale, v_scale): the inputs stand for scale * x8."""
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    q = torch.randn((batch, s_q, h_q, d), generator=g, dtype=torch.float32)
+    k = torch.randn((batch, s_k, h_kv, d), generator=g, dtype=torch.float32) * k_scale
+    v = torch.randn((batch, s_k, h_kv, d), generator=g, dtype=torch.float32)
+    out = []
+    scales = []
+    for t in (q, k, v):
+        sc = float(t.abs().max()) / 448.0
+        out.append((t / sc).to(torch.float8_e4m3fn))
+        scales.append(sc)
+    return (*out, *scales)

@@ -269,3 +269,15 @@ def test_bwd_entry_validation(lib):
     assert f(*a) == attn.ATTN_ERR_INVALID
     if not torch.cuda.is_available():
         assert f(*base) == attn.ATTN_ERR_CUDA
+
+
+def test_fp8_entry_validation(lib):
+    f = lib.attn_fwd_fp8
+    ok = (A, A, A, A, A, 1, 2, 2, 256, 256, 128, 0, 0.088)
+    assert f(*ok, float("nan"), 1.0, 1.0, None) == attn.ATTN_ERR_INVALID
+    assert f(*ok, 1.0, float("inf"), 1.0, None) == attn.ATTN_ERR_INVALID
+    assert f(*ok, 1.0, 1.0, float("nan"), None) == attn.ATTN_ERR_INVALID
+    assert f(*ok[:10], 64, 0, 0.088, 1.0, 1.0, 1.0, None) == attn.ATTN_ERR_UNSUPPORTED
+    assert f(A + 8, *ok[1:], 1.0, 1.0, 1.0, None) == attn.ATTN_ERR_ALIGN
+    if not torch.cuda.is_available():
+        assert f(*ok, 1.0, 1.0, 1.0, None) == attn.ATTN_ERR_CUDA

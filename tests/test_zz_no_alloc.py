@@ -5,8 +5,8 @@ handed only host arrays by an application owning all device memory, or code
 that cannot afford the synchronisation cudaMalloc/cudaFree may imply.  For
 them the library stages the copies in its own static device array.  This
 checks, through the C ABI, that two calls in a row give the same result as
-the workspace-taking entry point (attn_fwd_host), within the parity
-tolerances, and that oversized problems are refused.  Collected last so a
+the workspace-taking entry point (attn_fwd_host) and as the FP64 oracle,
+within the parity tolerances, and that oversized problems are refused.  Collected last so a
 stop-at-first-failure run has already run every other test.
 """
 from __future__ import annotations
@@ -17,6 +17,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 from parity import assert_within, gather_rows, metrics
 from scaled_dot_product_10_b200 import attn
 from scaled_dot_product_10_b200.workloads import make_qkv
@@ -63,14 +64,24 @@ def _workspace_call(q, k, v, causal):
 
 
 def test_static_entry_matches_workspace_entry_twice():
+    # Two calls in a row through the shared staging array (different sizes,
+    # so the second overwrites part of what the first left there); each
+    # result is then compared with the workspace-taking entry point and with
+    # the FP64 oracle, within the parity tolerances.
     cases = [((2, 4, 2, 513, 7100), True), ((1, 8, 1, 1000, 7101), False)]
+    runs = []
     for (b, hq, hkv, s, seed), causal in cases:
         q, k, v, o, lse = _pinned(b, hq, hkv, s, seed)
         _static_call(q, k, v, o, lse, causal)
-        o_ref, lse_ref = _workspace_call(q, k, v, causal)
+        runs.append((q, k, v, o, lse, causal))
+    for q, k, v, o, lse, causal in runs:
+        b, s = q.shape[0], q.shape[1]
+        o_ws, lse_ws = _workspace_call(q, k, v, causal)
         a, la = gather_rows(o, lse, None)
-        r, lr = gather_rows(o_ref, lse_ref, None)
+        r, lr = gather_rows(o_ws, lse_ws, None)
         assert_within(metrics(a, la, r, lr), f"static vs workspace b={b} s={s}")
+        o_ref, l_ref, _ = oracle.attn_fwd(q, k, v, causal, 1.0 / math.sqrt(q.shape[3]))
+        assert_within(metrics(a, la, o_ref, l_ref), f"static vs oracle b={b} s={s}")
 
 
 def test_static_entry_refuses_oversized_problem():
