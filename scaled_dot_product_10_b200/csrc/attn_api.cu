@@ -456,7 +456,7 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     p.section = p.num_items <= rounds4 ? batch * h_kv : kHeadsPerSection;
     if (p.section > batch * h_kv) p.section = batch * h_kv;
     int grid = p.num_items < st->num_sms ? p.num_items : st->num_sms;
-    bwd::dkdv::attn_bwd_dkdv_kernel<<<grid, bwd::kThreads, bwd::dkdv::Smem::kAlloc, cs>>>(
+    bwd::dkdv::attn_bwd_dkdv_kernel<<<grid, bwd::dkdv::kThreads, bwd::dkdv::Smem::kAlloc, cs>>>(
         tq64, tk, tv, tdo64, tdk, tdv, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
@@ -465,8 +465,8 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     p.section = p.num_items <= rounds4 ? batch * h_q : kHeadsPerSection;
     if (p.section > batch * h_q) p.section = batch * h_q;
     grid = p.num_items < st->num_sms ? p.num_items : st->num_sms;
-    bwd::dq::attn_bwd_dq_kernel<<<grid, bwd::kThreads, bwd::dq::Smem::kAlloc, cs>>>(tq, tk, tv,
-                                                                                     tdo, tdq, p);
+    bwd::dq::attn_bwd_dq_kernel<<<grid, bwd::dq::kThreads, bwd::dq::Smem::kAlloc, cs>>>(
+        tq, tk, tv, tdo, tdq, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
     g_last_launches = 3;
     return ATTN_OK;

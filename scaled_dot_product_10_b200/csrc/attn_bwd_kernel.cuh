@@ -14,17 +14,23 @@
 //   attn_bwd_prep_kernel  -- D and L per query row (memory-bound), written
 //                            to a padded workspace (padding rows: L = +inf,
 //                            D = 0, so they carry weight 0);
-//   attn_bwd_dq_kernel    -- one CTA per 128-row query block (persistent):
-//                            Q and dO stay in shared memory, K/V tiles
-//                            stream through a two-slot ring; per key block
-//                            S and dP on the tensor core (TMEM), dS by one
-//                            warpgroup, dQ += dS K on the tensor core;
-//   attn_bwd_dkdv_kernel  -- one CTA per 128-key block of a key/value head:
-//                            K and V stay in shared memory, 64-row Q/dO
-//                            tiles of every query head of the group stream
-//                            through; S^T = K Q^T and dP^T = V dO^T on the
-//                            tensor core, P^T and dS^T by one warpgroup
-//                            (thread = key), dV += P^T dO and dK += dS^T Q.
+//   attn_bwd_dq_kernel    -- one CTA item per 128-row query block
+//                            (persistent): Q and dO stay in shared memory,
+//                            K/V tiles stream through a two-slot ring; per
+//                            key block S and dP on the tensor core (TMEM),
+//                            dS by one warpgroup (thread = row), dQ += dS K
+//                            on the tensor core;
+//   attn_bwd_dkdv_kernel  -- one CTA item per 128-key block of a key/value
+//                            head: K and V stay in shared memory, 64-row
+//                            Q/dO tiles of every query head of the group
+//                            stream through a three-slot ring; S^T = K Q^T
+//                            and dP^T = V dO^T on the tensor core, P^T and
+//                            dS^T by one of two warpgroups (alternate steps,
+//                            thread = key), dV += P^T dO and dK += dS^T Q.
+// In the dK/dV kernel one warpgroup's exponentials run while the other's
+// products are on the tensor core.  (The same split for dQ, with 64-key
+// steps, measured slower on B200 than this single-warpgroup dQ kernel with
+// 128-key steps, which already overlaps S(j+1) with block j's softmax.)
 // Splitting dQ from dK/dV costs a second Q K^T and dO V^T but needs no
 // atomics: every output element is written once, by one CTA, and the result
 // is bit-for-bit reproducible.
@@ -36,9 +42,6 @@ namespace sdpa10 {
 namespace bwd {
 
 constexpr int kBlockQ = 64;             // query rows per dK/dV step
-constexpr int kThreads = 192;           // 4 compute warps, producer, MMA issuer
-constexpr int kLoadWarp = 4;
-constexpr int kMmaWarp = 5;
 constexpr int kQTile64Bytes = kBlockQ * kHeadDim * 2;  // 16 KiB: 64 rows x 128
 constexpr int kHalf64Bytes = kQTile64Bytes / 2;         // one 64-column half
 
@@ -127,6 +130,12 @@ __global__ void __launch_bounds__(kPrepThreads) attn_bwd_prep_kernel(const PrepP
 
 // ------------------------------------------------------------------ dQ kernel
 namespace dq {
+
+// One compute warpgroup (warps 0-3), the TMA producer (warp 4) and the MMA
+// issuer (warp 5).
+constexpr int kThreads = 192;
+constexpr int kLoadWarp = 4;
+constexpr int kMmaWarp = 5;
 
 struct Smem {
     static constexpr int kQ = 0;                       // Q tile  (A of S = Q K^T)
@@ -517,25 +526,40 @@ namespace sdpa10 {
 namespace bwd {
 namespace dkdv {
 
+// Two compute warpgroups take alternate 64-row steps (warps 0-3 the even
+// global steps, warps 4-7 the odd ones), so one warpgroup's exponentials and
+// dS^T run while the other's tiles are on the tensor core; warp 8 is the
+// TMA producer and warp 9 the MMA issuer.
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kQDStages = 3;
+
 struct Smem {
-    static constexpr int kK = 0;                                // K tile (A of S^T = K Q^T)
-    static constexpr int kV = kTileBytes;                       // V tile (A of dP^T = V dO^T)
-    static constexpr int kQD = 2 * kTileBytes;                  // ring of 2 x (Q 64 rows, dO 64 rows)
-    static constexpr int kQDSlot = 2 * kQTile64Bytes;           // 32 KiB per slot
-    static constexpr int kPT = kQD + 2 * kQDSlot;               // P^T  [128 keys x 64] (A of dV)
-    static constexpr int kDST = kPT + kQTile64Bytes;            // dS^T [128 keys x 64] (A of dK)
-    static constexpr int kStage = kDST + kQTile64Bytes;         // dK / dV store staging (32 KiB)
-    static constexpr int kLD = kStage + kTileBytes;             // ring of 2 x (L[64], D[64])
-    static constexpr int kBars = kLD + 2 * 512;
-    static constexpr int bKVFull = 0, bKVEmpty = 1, bQDFull = 2, bQDEmpty = 4, bSFull = 6,
-                         bSFree = 7, bPFull = 8, bPFree = 9, bPTFull = 10, bPTFree = 11,
-                         bDSTFull = 12, bDSTFree = 13, bAccFull = 14, bAccFree = 15,
-                         bStaged = 16, bStored = 17, bDrain = 18, kNumBars = 19;
+    static constexpr int kK = 0;                              // K tile (A of S^T = K Q^T)
+    static constexpr int kV = kTileBytes;                     // V tile (A of dP^T = V dO^T)
+    static constexpr int kQD = 2 * kTileBytes;                // ring of 3 x (Q 64 rows, dO 64 rows)
+    static constexpr int kQDSlot = 2 * kQTile64Bytes;         // 32 KiB per slot
+    // Per warpgroup w: P^T_w then dS^T_w ([128 keys x 64], 16 KiB each),
+    // 32 KiB contiguous; at the end of an item warpgroup 0 stages dV and
+    // warpgroup 1 stages dK there for the TMA store.
+    static constexpr int kWG = kQD + kQDStages * kQDSlot;
+    static constexpr int kWGBytes = 2 * kQTile64Bytes;
+    static constexpr int kLD = kWG + 2 * kWGBytes;            // ring of 3 x (L[64], D[64])
+    static constexpr int kBars = kLD + kQDStages * 512;
+    static constexpr int bKVFull = 0, bKVEmpty = 1, bQDFull = 2, bQDEmpty = 2 + kQDStages,
+                         bSFull = 2 + 2 * kQDStages,       // [2] per warpgroup from here on
+                         bSFree = bSFull + 2, bPFull = bSFree + 2, bPFree = bPFull + 2,
+                         bPTFull = bPFree + 2, bPTFree = bPTFull + 2, bDSTFull = bPTFree + 2,
+                         bDSTFree = bDSTFull + 2, bStaged = bDSTFree + 2, bStored = bStaged + 2,
+                         bAccFull = bStored + 2, bAccFree = bAccFull + 1, bDrain = bAccFree + 1,
+                         kNumBars = bDrain + 1;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
     static constexpr int kBytes = kAbort + 4;
     static constexpr int kAlloc = kBytes + 1024;
 };
+static_assert(Smem::kAlloc <= 232448, "dK/dV shared memory exceeds the per-CTA limit");
 
 // Item t -> (key block, batch, key/value head): by section of heads, then
 // key block ascending (under the causal mask the first key blocks are seen
@@ -602,28 +626,29 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
     volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
-
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
         ptx::mbar_init(bar(L::bKVFull), 1);
         ptx::mbar_init(bar(L::bKVEmpty), 1);
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < kQDStages; ++i) {
             ptx::mbar_init(bar(L::bQDFull + i), 1);
             ptx::mbar_init(bar(L::bQDEmpty + i), 1);
         }
-        ptx::mbar_init(bar(L::bSFull), 1);
-        ptx::mbar_init(bar(L::bSFree), 4);
-        ptx::mbar_init(bar(L::bPFull), 1);
-        ptx::mbar_init(bar(L::bPFree), 4);
-        ptx::mbar_init(bar(L::bPTFull), 4);
-        ptx::mbar_init(bar(L::bPTFree), 1);
-        ptx::mbar_init(bar(L::bDSTFull), 4);
-        ptx::mbar_init(bar(L::bDSTFree), 1);
+        for (int w = 0; w < 2; ++w) {
+            ptx::mbar_init(bar(L::bSFull + w), 1);
+            ptx::mbar_init(bar(L::bSFree + w), 4);
+            ptx::mbar_init(bar(L::bPFull + w), 1);
+            ptx::mbar_init(bar(L::bPFree + w), 4);
+            ptx::mbar_init(bar(L::bPTFull + w), 4);
+            ptx::mbar_init(bar(L::bPTFree + w), 1);
+            ptx::mbar_init(bar(L::bDSTFull + w), 4);
+            ptx::mbar_init(bar(L::bDSTFree + w), 1);
+            ptx::mbar_init(bar(L::bStaged + w), 4);
+            ptx::mbar_init(bar(L::bStored + w), 1);
+        }
         ptx::mbar_init(bar(L::bAccFull), 1);
-        ptx::mbar_init(bar(L::bAccFree), 4);
-        ptx::mbar_init(bar(L::bStaged), 4);
-        ptx::mbar_init(bar(L::bStored), 1);
+        ptx::mbar_init(bar(L::bAccFree), 8);  // both warpgroups have read dV / dK
         ptx::mbar_init(bar(L::bDrain), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
@@ -643,9 +668,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    // TMEM: S^T | dP^T (64 columns each) | dV | dK at columns 0, 64, 128, 256.
+    // TMEM: S^T_0 | S^T_1 | dP^T_0 | dP^T_1 (64 columns each) | dV | dK at
+    // columns 0, 64, 128, 192, 256, 384.
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
+    auto qd_addr = [&](uint32_t u) { return sbase + L::kQD + (u % kQDStages) * L::kQDSlot; };
 
     if (warp == kLoadWarp) {
         // ============================================================ producer
@@ -671,11 +698,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const int hl = s / c.nq;
                     const int qb = c.qlo + (s - hl * c.nq);
                     const int h = c.g * p.group + hl;
-                    const uint32_t slot = qd_loads & 1;
-                    if (!(ok = wait_bar(bar(L::bQDEmpty + slot), ((qd_loads >> 1) & 1) ^ 1, wc)))
+                    const uint32_t slot = qd_loads % kQDStages;
+                    if (!(ok = wait_bar(bar(L::bQDEmpty + slot),
+                                        ((qd_loads / kQDStages) & 1) ^ 1, wc)))
                         break;
                     const uint32_t full = bar(L::bQDFull + slot);
-                    const uint32_t dst = sbase + L::kQD + slot * L::kQDSlot;
+                    const uint32_t dst = qd_addr(qd_loads);
                     ptx::mbar_arrive_expect_tx(full, 2 * kQTile64Bytes + 512);
 #pragma unroll
                     for (int half = 0; half < 2; ++half) {
@@ -692,9 +720,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             if (kv_loads > 0) wait_slow(bar(L::bKVFull), (kv_loads - 1) & 1, wc, false);
-            for (int i = 0; i < 2 && i < static_cast<int>(qd_loads); ++i) {
+            for (int i = 0; i < kQDStages && i < static_cast<int>(qd_loads); ++i) {
                 const uint32_t f = qd_loads - 1 - i;
-                wait_slow(bar(L::bQDFull + (f & 1)), (f >> 1) & 1, wc, false);
+                wait_slow(bar(L::bQDFull + f % kQDStages), (f / kQDStages) & 1, wc, false);
             }
         }
         __syncwarp();
@@ -705,10 +733,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t kIdAcc = idesc_bf16_f32(kBlockN, kHeadDim, 0, 1);  // P^T dO, dS^T Q
             const uint32_t k_lo = desc_lo_sw128(sbase + L::kK, 16);
             const uint32_t v_lo = desc_lo_sw128(sbase + L::kV, 16);
-            const uint32_t pt_lo = desc_lo_sw128(sbase + L::kPT, 16);
-            const uint32_t dst_lo = desc_lo_sw128(sbase + L::kDST, 16);
-            const uint32_t s_tm = tmem, dp_tm = tmem + 64, dv_tm = tmem + 128, dk_tm = tmem + 256;
-            uint32_t items = 0, qd_used = 0, step_all = 0;
+            const uint32_t dv_tm = tmem + 256, dk_tm = tmem + 384;
+            uint32_t items = 0, gs0 = 0;
             bool ok = true;
             // X^T = A B^T with A a [128 x 128] K-major tile (K or V) and B a
             // 64-row K-major tile (Q or dO): 8 K-steps; the 64-row tile's
@@ -733,50 +759,53 @@ __global__ void __launch_bounds__(kThreads, 1)
                                 desc_from_lo(b_lo + ((k * 2048) >> 4)), kIdAcc,
                                 (acc || k > 0) ? 1u : 0u);
             };
-            auto qd_addr = [&](uint32_t u) { return sbase + L::kQD + (u & 1) * L::kQDSlot; };
+            // S^T and dP^T of global step gs into warpgroup (gs & 1)'s
+            // columns once that warpgroup has read its previous ones.
+            auto scores = [&](uint32_t gs) -> bool {
+                const uint32_t w = gs & 1, i = gs >> 1;
+                if (!wait_bar(bar(L::bQDFull + gs % kQDStages), (gs / kQDStages) & 1, wc))
+                    return false;
+                if (i > 0 && !wait_bar(bar(L::bSFree + w), (i - 1) & 1, wc)) return false;
+                ptx::tc_fence_after();
+                gemm_t(tmem + 64 * w, k_lo, desc_lo_sw128(qd_addr(gs), 16));
+                ptx::mma_commit(bar(L::bSFull + w));
+                if (i > 0 && !wait_bar(bar(L::bPFree + w), (i - 1) & 1, wc)) return false;
+                ptx::tc_fence_after();
+                gemm_t(tmem + 128 + 64 * w, v_lo, desc_lo_sw128(qd_addr(gs) + kQTile64Bytes, 16));
+                ptx::mma_commit(bar(L::bPFull + w));
+                return true;
+            };
             Cursor c;
             for (c.start(p); ok && c.valid(p); c.next(p)) {
                 const int n = c.steps(p);
                 if (!(ok = wait_bar(bar(L::bKVFull), items & 1, wc))) break;
+                // Per item: S^T, dP^T of its first two steps, then per step
+                // s: dV(s), dK(s), then S^T, dP^T of step s + 2 (same
+                // warpgroup) -- the other warpgroup's step s + 1 runs on the
+                // tensor core while this one's exponentials run.
+                if (!(ok = scores(gs0))) break;
+                if (n > 1 && !(ok = scores(gs0 + 1))) break;
                 // dV / dK of the previous item must have been read out.
                 if (items > 0 && !(ok = wait_bar(bar(L::bAccFree), (items - 1) & 1, wc))) break;
                 ++items;
-                // S^T(0) and dP^T(0), then per step s: S^T(s+1), dV(s),
-                // dP^T(s+1), dK(s) -- the next scores run under this step's
-                // exponentials.
-                auto scores = [&](uint32_t u, uint32_t gs) -> bool {
-                    if (!wait_bar(bar(L::bQDFull + (u & 1)), (u >> 1) & 1, wc)) return false;
-                    if (gs > 0 && !wait_bar(bar(L::bSFree), (gs - 1) & 1, wc)) return false;
-                    ptx::tc_fence_after();
-                    gemm_t(s_tm, k_lo, desc_lo_sw128(qd_addr(u), 16));
-                    ptx::mma_commit(bar(L::bSFull));
-                    return true;
-                };
-                auto dprobs = [&](uint32_t u, uint32_t gs) -> bool {
-                    if (gs > 0 && !wait_bar(bar(L::bPFree), (gs - 1) & 1, wc)) return false;
-                    ptx::tc_fence_after();
-                    gemm_t(dp_tm, v_lo, desc_lo_sw128(qd_addr(u) + kQTile64Bytes, 16));
-                    ptx::mma_commit(bar(L::bPFull));
-                    return true;
-                };
-                if (!(ok = scores(qd_used, step_all) && dprobs(qd_used, step_all))) break;
                 for (int s = 0; s < n && ok; ++s) {
-                    const uint32_t u = qd_used + s, gs = step_all + s;
-                    if (s + 1 < n && !(ok = scores(u + 1, gs + 1))) break;
-                    if (!(ok = wait_bar(bar(L::bPTFull), gs & 1, wc))) break;
+                    const uint32_t gs = gs0 + s, w = gs & 1, i = gs >> 1;
+                    const uint32_t pt_lo = desc_lo_sw128(sbase + L::kWG + w * L::kWGBytes, 16);
+                    const uint32_t dst_lo =
+                        desc_lo_sw128(sbase + L::kWG + w * L::kWGBytes + kQTile64Bytes, 16);
+                    if (!(ok = wait_bar(bar(L::bPTFull + w), i & 1, wc))) break;
                     ptx::tc_fence_after();
-                    gemm_acc(dv_tm, pt_lo, qd_addr(u) + kQTile64Bytes, s > 0);
-                    ptx::mma_commit(bar(L::bPTFree));
-                    if (s + 1 < n && !(ok = dprobs(u + 1, gs + 1))) break;
-                    if (!(ok = wait_bar(bar(L::bDSTFull), gs & 1, wc))) break;
+                    gemm_acc(dv_tm, pt_lo, qd_addr(gs) + kQTile64Bytes, s > 0);
+                    ptx::mma_commit(bar(L::bPTFree + w));
+                    if (!(ok = wait_bar(bar(L::bDSTFull + w), i & 1, wc))) break;
                     ptx::tc_fence_after();
-                    gemm_acc(dk_tm, dst_lo, qd_addr(u), s > 0);
-                    ptx::mma_commit(bar(L::bDSTFree));
-                    ptx::mma_commit(bar(L::bQDEmpty + (u & 1)));
+                    gemm_acc(dk_tm, dst_lo, qd_addr(gs), s > 0);
+                    ptx::mma_commit(bar(L::bDSTFree + w));
+                    ptx::mma_commit(bar(L::bQDEmpty + gs % kQDStages));
+                    if (s + 2 < n && !(ok = scores(gs + 2))) break;
                 }
                 if (!ok) break;
-                qd_used += n;
-                step_all += n;
+                gs0 += n;
                 ptx::mma_commit(bar(L::bKVEmpty));
                 ptx::mma_commit(bar(L::bAccFull));
             }
@@ -786,24 +815,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ============================================================ compute
-        // Thread r owns key row r of the block (TMEM lane r).
-        const int r = warp * 32 + lane;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t s_tm = tmem + lane_base, dp_tm = tmem + lane_base + 64,
-                       dv_tm = tmem + lane_base + 128, dk_tm = tmem + lane_base + 256;
+        // Warpgroup w = warp / 4; thread r owns key row r of the block (TMEM
+        // lane r) and takes the global steps gs with gs % 2 == w.
+        const int w = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t s_tm = tmem + lane_base + 64 * w, dp_tm = tmem + lane_base + 128 + 64 * w;
+        const uint32_t acc_tm = tmem + lane_base + (w ? 384 : 256);  // dK (w 1) or dV (w 0)
         // Row r of a [128 x 64] K-major tile: 8 chunks of 16 bytes, chunk cc
         // at (r / 8) * 1024 + (r % 8) * 128 + ((cc ^ (r % 8)) * 16).
         const uint32_t xr = static_cast<uint32_t>(r & 7);
-        const uint32_t pt_row = sbase + L::kPT + (r >> 3) * 1024 + (r & 7) * 128;
-        const uint32_t dst_row = sbase + L::kDST + (r >> 3) * 1024 + (r & 7) * 128;
-        const uint32_t st_row = sbase + L::kStage + (r >> 3) * 1024 + (r & 7) * 128;
+        const uint32_t wg_base = sbase + L::kWG + w * L::kWGBytes;
+        const uint32_t row_off = (r >> 3) * 1024 + (r & 7) * 128;
+        const uint32_t pt_row = wg_base + row_off;
+        const uint32_t dst_row = wg_base + kQTile64Bytes + row_off;
+        const uint32_t st_row = wg_base + row_off;  // [128 x 128] staging, halves 16 KiB apart
         const float c2 = p.scale_log2;
-        uint32_t items = 0, gs = 0;
+        uint32_t items = 0, gs0 = 0, mine = 0;  // mine: steps this warpgroup has done
         Cursor c;
         for (c.start(p); c.valid(p); c.next(p)) {
             const int n = c.steps(p);
             const int key = c.kb * kBlockN + r;
-            for (int s = 0; s < n; ++s, ++gs) {
+            for (int s = (gs0 & 1) == static_cast<uint32_t>(w) ? 0 : 1; s < n; s += 2, ++mine) {
+                const uint32_t gs = gs0 + s;
                 const int hl = s / c.nq;
                 const int qb = c.qlo + (s - hl * c.nq);
                 // Visible query columns of this key row: [lo, hi].
@@ -811,15 +845,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (p.causal) lo = key - p.causal_offset - qb * kBlockQ;
                 if (p.window_left >= 0)
                     hi = min(hi, key + p.window_left - p.causal_offset - qb * kBlockQ);
-                const uint32_t slot = gs & 1;
+                const uint32_t slot = gs % kQDStages;
                 const uint32_t sL = sbase + L::kLD + slot * 512;  // L[64], then D[64]
                 const uint32_t sD = sL + 256;
                 float pt[64];
                 // L and D of this step's rows arrive with its Q / dO tiles
                 // (the slot is refilled only after this step's dK MMA, which
                 // waits for this warpgroup).
-                if (!wait_bar_warp(bar(L::bQDFull + slot), (gs >> 1) & 1, wc)) return;
-                if (!wait_bar_warp(bar(L::bSFull), gs & 1, wc)) return;
+                if (!wait_bar_warp(bar(L::bQDFull + slot), (gs / kQDStages) & 1, wc)) return;
+                if (!wait_bar_warp(bar(L::bSFull + w), mine & 1, wc)) return;
                 ptx::tc_fence_after();
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
@@ -831,7 +865,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(L::bSFree));
+                if (lane == 0) ptx::mbar_arrive(bar(L::bSFree + w));
 #pragma unroll
                 for (int k4 = 0; k4 < 16; ++k4) {
                     const float4 l4 = ptx::ld_shared_f4(sL + 16 * k4);  // same address: broadcast
@@ -843,8 +877,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pt[k] = (k >= lo && k <= hi) ? x : 0.f;
                     }
                 }
-                // P^T -> BF16 into its tile once the last dV MMA has read it.
-                if (gs > 0 && !wait_bar_warp(bar(L::bPTFree), (gs - 1) & 1, wc)) return;
+                // P^T -> BF16 into this warpgroup's tile once its last dV
+                // MMA has read it.
+                if (mine > 0 && !wait_bar_warp(bar(L::bPTFree + w), (mine - 1) & 1, wc)) return;
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc)
                     ptx::st_shared_v4(pt_row + ((cc ^ xr) << 4),
@@ -854,10 +889,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       ptx::pack_bf16x2(pt[8 * cc + 6], pt[8 * cc + 7]));
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(L::bPTFull));
+                if (lane == 0) ptx::mbar_arrive(bar(L::bPTFull + w));
                 // dS^T = P^T (dP^T - D) -> BF16.
-                if (!wait_bar_warp(bar(L::bPFull), gs & 1, wc)) return;
-                if (gs > 0 && !wait_bar_warp(bar(L::bDSTFree), (gs - 1) & 1, wc)) return;
+                if (!wait_bar_warp(bar(L::bPFull + w), mine & 1, wc)) return;
+                if (mine > 0 && !wait_bar_warp(bar(L::bDSTFree + w), (mine - 1) & 1, wc)) return;
                 ptx::tc_fence_after();
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
@@ -877,7 +912,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(L::bPFree));
+                if (lane == 0) ptx::mbar_arrive(bar(L::bPFree + w));
 #pragma unroll
                 for (int cc = 0; cc < 8; ++cc)
                     ptx::st_shared_v4(dst_row + ((cc ^ xr) << 4),
@@ -887,55 +922,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                                       ptx::pack_bf16x2(pt[8 * cc + 6], pt[8 * cc + 7]));
                 ptx::fence_proxy_async_smem();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(L::bDSTFull));
+                if (lane == 0) ptx::mbar_arrive(bar(L::bDSTFull + w));
             }
-            // Epilogue: dV, then dK * scale, as BF16 rows staged in the
-            // [128 x 128] staging tile and stored with TMA (rows past s_k are
-            // clipped by the tensor map).
+            gs0 += n;
+            // Epilogue: warpgroup 0 writes dV, warpgroup 1 dK * scale, as
+            // BF16 rows staged in its own 32 KiB (its P^T and dS^T tiles, free
+            // once every MMA of the item has completed) and stored with TMA
+            // (rows past s_k are clipped by the tensor map).
             if (!wait_bar_warp(bar(L::bAccFull), items & 1, wc)) return;
             ptx::tc_fence_after();
-#pragma unroll 1
-            for (int which = 0; which < 2; ++which) {
-                const uint32_t src = which ? dk_tm : dv_tm;
-                const float f = which ? p.scale : 1.f;
+            const float f = w ? p.scale : 1.f;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    uint32_t v[32];
-                    ptx::tmem_ld32(src + q * 32, v);
-                    ptx::tmem_wait_ld();
+            for (int q = 0; q < 4; ++q) {
+                uint32_t v[32];
+                ptx::tmem_ld32(acc_tm + q * 32, v);
+                ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int cc = 4 * q + k;
-                        ptx::st_shared_v4(
-                            st_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ xr) << 4),
-                            ptx::pack_bf16x2(__uint_as_float(v[8 * k]) * f, __uint_as_float(v[8 * k + 1]) * f),
-                            ptx::pack_bf16x2(__uint_as_float(v[8 * k + 2]) * f, __uint_as_float(v[8 * k + 3]) * f),
-                            ptx::pack_bf16x2(__uint_as_float(v[8 * k + 4]) * f, __uint_as_float(v[8 * k + 5]) * f),
-                            ptx::pack_bf16x2(__uint_as_float(v[8 * k + 6]) * f, __uint_as_float(v[8 * k + 7]) * f));
-                    }
+                for (int k = 0; k < 4; ++k) {
+                    const int cc = 4 * q + k;
+                    ptx::st_shared_v4(
+                        st_row + (cc >> 3) * kQTile64Bytes + (((cc & 7) ^ xr) << 4),
+                        ptx::pack_bf16x2(__uint_as_float(v[8 * k]) * f, __uint_as_float(v[8 * k + 1]) * f),
+                        ptx::pack_bf16x2(__uint_as_float(v[8 * k + 2]) * f, __uint_as_float(v[8 * k + 3]) * f),
+                        ptx::pack_bf16x2(__uint_as_float(v[8 * k + 4]) * f, __uint_as_float(v[8 * k + 5]) * f),
+                        ptx::pack_bf16x2(__uint_as_float(v[8 * k + 6]) * f, __uint_as_float(v[8 * k + 7]) * f));
                 }
-                if (which == 1) {
-                    ptx::tc_fence_before();
-                }
-                ptx::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) {
-                    if (which == 1) ptx::mbar_arrive(bar(L::bAccFree));
-                    ptx::mbar_arrive(bar(L::bStaged));
-                }
-                const uint32_t ph = (2 * items + which) & 1;
-                if (r == 0) {
-                    if (!wait_bar(bar(L::bStaged), ph, wc)) return;
-                    const CUtensorMap* tm = which ? &tm_dk : &tm_dv;
-                    ptx::tma_store_4d(tm, sbase + L::kStage, 0, c.g, c.kb * kBlockN, c.b);
-                    ptx::tma_store_4d(tm, sbase + L::kStage + kHalfTileBytes, 64, c.g,
-                                      c.kb * kBlockN, c.b);
-                    ptx::bulk_commit_group();
-                    ptx::bulk_wait_group_read0();
-                    ptx::mbar_arrive(bar(L::bStored));
-                }
-                if (!wait_bar_warp(bar(L::bStored), ph, wc)) return;
             }
+            ptx::tc_fence_before();
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+                ptx::mbar_arrive(bar(L::bAccFree));
+                ptx::mbar_arrive(bar(L::bStaged + w));
+            }
+            if (r == 0) {
+                if (!wait_bar(bar(L::bStaged + w), items & 1, wc)) return;
+                const CUtensorMap* tm = w ? &tm_dk : &tm_dv;
+                ptx::tma_store_4d(tm, wg_base, 0, c.g, c.kb * kBlockN, c.b);
+                ptx::tma_store_4d(tm, wg_base + kQTile64Bytes, 64, c.g, c.kb * kBlockN, c.b);
+                ptx::bulk_commit_group();
+                ptx::bulk_wait_group_read0();
+                ptx::mbar_arrive(bar(L::bStored + w));
+            }
+            // This warpgroup's tiles are rewritten by its next step only
+            // after TMA has read the staged rows.
+            if (!wait_bar_warp(bar(L::bStored + w), items & 1, wc)) return;
             ++items;
         }
         if (r == 0) ptx::bulk_wait_group0();
