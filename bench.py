@@ -81,17 +81,31 @@ def kernel_source_hash() -> str:
     return h.hexdigest()[:16]
 
 
+FWD_SOURCES = ("attn_fwd_kernel.cuh", "attn_common.cuh", "sm100_ptx.cuh", "attn_api.cu")
+
+
+def fwd_kernel_hash() -> str:
+    """Hash of the sources the forward kernel and its launch are built from."""
+    h = hashlib.sha256()
+    for name in FWD_SOURCES:
+        with open(os.path.join(ROOT, "scaled_dot_product_10_b200", "csrc", name), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
 def committed_traffic(workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel sources; else None."""
+    """DRAM bytes per launch of the forward on this workload from the
+    committed ncu capture (profiles/traffic.json), if it was taken on the
+    current forward sources; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
     with open(path) as f:
         d = json.load(f)
-    if d.get("kernel_hash") != kernel_source_hash() or d.get("workload") != workload:
+    entry = d.get("workloads", {}).get(workload)
+    if not entry or entry.get("fwd_kernel_hash") != fwd_kernel_hash():
         return None
-    return d.get("dram_bytes_per_launch")
+    return entry.get("dram_bytes_per_launch")
 
 
 class ClockSampler:
@@ -378,6 +392,7 @@ def run_ours(args, world, rank, local):
         "clocks": sampler.summary(),
         "gpu_launches": 2 * K,
         "kernel_hash": kernel_source_hash(),
+        "fwd_kernel_hash": fwd_kernel_hash(),
     }
 
     if not args.no_e2e:
