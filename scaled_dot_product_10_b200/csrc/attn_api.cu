@@ -92,11 +92,48 @@ int init_device(int dev, DeviceState** out) {
     return ATTN_OK;
 }
 
+// Encoded tensor maps of recent calls, per host thread: a map depends only
+// on its base address, shape, element type and box, so a call that repeats
+// a tensor (the usual case in a loop) reuses it instead of encoding it again
+// on the launch path.
+struct MapKey {
+    const void* base;
+    int heads, seq, batch, box_rows, fp8;
+    bool operator==(const MapKey& o) const {
+        return base == o.base && heads == o.heads && seq == o.seq && batch == o.batch &&
+               box_rows == o.box_rows && fp8 == o.fp8;
+    }
+};
+constexpr int kMapCacheSize = 16;
+struct MapCache {
+    MapKey key[kMapCacheSize];
+    CUtensorMap map[kMapCacheSize];
+    int used = 0, next = 0;
+};
+thread_local MapCache g_map_cache;
+
+bool cached_map(CUtensorMap* m, const MapKey& k, bool (*encode)(CUtensorMap*, const MapKey&)) {
+    MapCache& c = g_map_cache;
+    for (int i = 0; i < c.used; ++i)
+        if (c.key[i] == k) {
+            *m = c.map[i];
+            return true;
+        }
+    if (!encode(m, k)) return false;
+    c.key[c.next] = k;
+    c.map[c.next] = *m;
+    c.next = (c.next + 1) % kMapCacheSize;
+    if (c.used < kMapCacheSize) ++c.used;
+    return true;
+}
+
 // [batch, seq, heads, 128] BF16 as a 4-D tensor map {d, heads, seq, batch},
 // box {64, 1, box_rows, 1} (one 128-byte swizzled half of a box_rows-row
 // tile; 128 rows unless given).
-bool encode_map(CUtensorMap* m, const void* base, int heads, int seq, int batch,
-                unsigned box_rows = 128) {
+bool encode_map_bf16(CUtensorMap* m, const MapKey& k) {
+    const void* base = k.base;
+    const int heads = k.heads, seq = k.seq, batch = k.batch;
+    const unsigned box_rows = static_cast<unsigned>(k.box_rows);
     cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(heads),
                           static_cast<cuuint64_t>(seq), static_cast<cuuint64_t>(batch)};
     cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHeadDim) * 2,
@@ -114,7 +151,9 @@ bool encode_map(CUtensorMap* m, const void* base, int heads, int seq, int batch,
 // [batch, seq, heads, 128] FP8 (one byte per element) as a 4-D tensor map,
 // box {128, 1, 128, 1}: a 128-row tile whose 128-byte rows are one swizzle
 // atom each.
-bool encode_map_fp8(CUtensorMap* m, const void* base, int heads, int seq, int batch) {
+bool encode_map_e4m3(CUtensorMap* m, const MapKey& k) {
+    const void* base = k.base;
+    const int heads = k.heads, seq = k.seq, batch = k.batch;
     cuuint64_t dims[4] = {static_cast<cuuint64_t>(kHeadDim), static_cast<cuuint64_t>(heads),
                           static_cast<cuuint64_t>(seq), static_cast<cuuint64_t>(batch)};
     cuuint64_t strides[3] = {static_cast<cuuint64_t>(kHeadDim),
@@ -127,6 +166,15 @@ bool encode_map_fp8(CUtensorMap* m, const void* base, int heads, int seq, int ba
                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
+}
+
+bool encode_map(CUtensorMap* m, const void* base, int heads, int seq, int batch,
+                int box_rows = 128) {
+    return cached_map(m, MapKey{base, heads, seq, batch, box_rows, 0}, encode_map_bf16);
+}
+
+bool encode_map_fp8(CUtensorMap* m, const void* base, int heads, int seq, int batch) {
+    return cached_map(m, MapKey{base, heads, seq, batch, 128, 1}, encode_map_e4m3);
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
