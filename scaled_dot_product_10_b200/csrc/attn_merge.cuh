@@ -34,6 +34,7 @@ struct MergeParams {
 };
 
 constexpr int kMergeThreads = 256;
+constexpr int kMergeBatch = 8;  // partials whose loads are in flight together
 
 __global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const MergeParams m) {
     const int lane = threadIdx.x & 31;
@@ -50,22 +51,45 @@ __global__ void __launch_bounds__(kMergeThreads) attn_merge_kernel(const MergePa
             nv = min(nv, (m.s_k + m.keys_per_part - 1) / m.keys_per_part);
             if (m.causal) nv = min(nv, (i + m.causal_offset) / m.keys_per_part + 1);
         }
+        // The loads of kMergeBatch partials are issued before any of them
+        // is combined (the row's partials are independent loads; walking
+        // them one by one left the kernel latency-bound).  The sums run in
+        // partial order, as the definition's left-to-right sum.
         float mx = -CUDART_INF_F;
-        for (int s = 0; s < nv; ++s) mx = fmaxf(mx, m.lse_part[static_cast<size_t>(s) * rows + r]);
+        for (int s0 = 0; s0 < nv; s0 += kMergeBatch) {
+            float l[kMergeBatch];
+#pragma unroll
+            for (int k = 0; k < kMergeBatch; ++k)
+                l[k] = s0 + k < nv ? m.lse_part[static_cast<size_t>(s0 + k) * rows + r]
+                                   : -CUDART_INF_F;
+#pragma unroll
+            for (int k = 0; k < kMergeBatch; ++k) mx = fmaxf(mx, l[k]);
+        }
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
         float wsum = 0.f;
         if (mx != -CUDART_INF_F) {
-            for (int s = 0; s < nv; ++s) {
-                const size_t idx = static_cast<size_t>(s) * rows + r;
-                const float l_s = m.lse_part[idx];
-                if (l_s == -CUDART_INF_F) continue;  // no keys: its O is not read
-                const float w = expf(l_s - mx);
-                const float4 v = reinterpret_cast<const float4*>(m.o_part + idx * 128)[lane];
-                wsum += w;
-                acc.x += w * v.x;
-                acc.y += w * v.y;
-                acc.z += w * v.z;
-                acc.w += w * v.w;
+            for (int s0 = 0; s0 < nv; s0 += kMergeBatch) {
+                float l[kMergeBatch];
+                float4 v[kMergeBatch];
+#pragma unroll
+                for (int k = 0; k < kMergeBatch; ++k) {
+                    const size_t idx = static_cast<size_t>(s0 + k) * rows + r;
+                    l[k] = s0 + k < nv ? m.lse_part[idx] : -CUDART_INF_F;
+                    // A part with no keys for the row (-inf) is not read.
+                    v[k] = l[k] != -CUDART_INF_F
+                               ? reinterpret_cast<const float4*>(m.o_part + idx * 128)[lane]
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
+#pragma unroll
+                for (int k = 0; k < kMergeBatch; ++k) {
+                    if (l[k] == -CUDART_INF_F) continue;
+                    const float w = expf(l[k] - mx);
+                    wsum += w;
+                    acc.x += w * v[k].x;
+                    acc.y += w * v[k].y;
+                    acc.z += w * v[k].z;
+                    acc.w += w * v[k].w;
+                }
             }
         }
         const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
