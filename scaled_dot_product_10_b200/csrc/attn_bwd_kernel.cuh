@@ -18,8 +18,9 @@
 //                            (persistent): Q and dO stay in shared memory,
 //                            K/V tiles stream through a two-slot ring; per
 //                            key block S and dP on the tensor core (TMEM),
-//                            dS by one warpgroup (thread = row), dQ += dS K
-//                            on the tensor core;
+//                            dS by two warpgroups (each 64 of the block's
+//                            keys, thread = row), dQ += dS K on the tensor
+//                            core;
 //   attn_bwd_dkdv_kernel  -- one CTA item per 128-key block of a key/value
 //                            head: K and V stay in shared memory, 64-row
 //                            Q/dO tiles of every query head of the group
@@ -131,11 +132,13 @@ __global__ void __launch_bounds__(kPrepThreads) attn_bwd_prep_kernel(const PrepP
 // ------------------------------------------------------------------ dQ kernel
 namespace dq {
 
-// One compute warpgroup (warps 0-3), the TMA producer (warp 4) and the MMA
-// issuer (warp 5).
-constexpr int kThreads = 192;
-constexpr int kLoadWarp = 4;
-constexpr int kMmaWarp = 5;
+// Two compute warpgroups (warps 0-3 and 4-7) split each 128-key step by
+// columns: warpgroup w takes keys 64w .. 64w + 63 of every row, so each row's
+// exponentials and dS run on two warps per SM sub-partition; warp 8 is the
+// TMA producer and warp 9 the MMA issuer.
+constexpr int kThreads = 320;
+constexpr int kLoadWarp = 8;
+constexpr int kMmaWarp = 9;
 
 struct Smem {
     static constexpr int kQ = 0;                       // Q tile  (A of S = Q K^T)
@@ -224,14 +227,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::mbar_init(bar(L::bVEmpty + i), 1);
         }
         ptx::mbar_init(bar(L::bSFull), 1);
-        ptx::mbar_init(bar(L::bSFree), 4);
+        ptx::mbar_init(bar(L::bSFree), 8);  // both compute warpgroups, 4 warps each
         ptx::mbar_init(bar(L::bPFull), 1);   // dP in TMEM
-        ptx::mbar_init(bar(L::bPFree), 4);
-        ptx::mbar_init(bar(L::bDsFull), 4);
+        ptx::mbar_init(bar(L::bPFree), 8);
+        ptx::mbar_init(bar(L::bDsFull), 8);
         ptx::mbar_init(bar(L::bDsFree), 1);
         ptx::mbar_init(bar(L::bDqFull), 1);
-        ptx::mbar_init(bar(L::bDqFree), 4);
-        ptx::mbar_init(bar(L::bStaged), 4);
+        ptx::mbar_init(bar(L::bDqFree), 8);
+        ptx::mbar_init(bar(L::bStaged), 8);
         ptx::mbar_init(bar(L::bStored), 1);
         ptx::mbar_init(bar(L::bDrain), 1);
         *abort_flag = 0;
@@ -391,12 +394,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ============================================================ compute
-        // Thread r owns query row r of the block (TMEM lane r).
-        const int r = warp * 32 + lane;
-        const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-        const uint32_t s_tm = tmem + lane_base, dp_tm = tmem + lane_base + 128,
-                       dq_tm = tmem + lane_base + 256;
-        const uint32_t ds_row = sbase + L::kDS + (r >> 3) * 1024 + (r & 7) * 128;
+        // Warpgroup `half` = warp / 4 takes columns 64 half .. 64 half + 63 of S, dP, dS
+        // and dQ; thread r owns query row r of the block (TMEM lane r).
+        const int half = warp >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t s_tm = tmem + lane_base + 64 * half,
+                       dp_tm = tmem + lane_base + 128 + 64 * half,
+                       dq_tm = tmem + lane_base + 256 + 64 * half;
+        // This row's half of the dS tile: the tile's 64-column half `half`
+        // (16 KiB), chunk k of the half at ((k ^ (r % 8)) * 16).
+        const uint32_t ds_row =
+            sbase + L::kDS + half * kHalfTileBytes + (r >> 3) * 1024 + (r & 7) * 128;
         const uint32_t xr = static_cast<uint32_t>(r & 7);
         const float c2 = p.scale_log2;
         uint32_t items = 0, steps = 0;
@@ -407,17 +416,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float Lr = p.L[stat];  // +inf past s_q: P = 0
             const float Dr = p.D[stat];
             for (int j = 0; j < c.n; ++j, ++steps) {
-                const int kv0 = (c.kb_lo + j) * kBlockN;
+                const int kv0 = (c.kb_lo + j) * kBlockN + 64 * half;  // this half's first key
                 // Visible keys of this row inside the block: [lo, hi).
-                int hi = min(kBlockN, p.s_k - kv0);
+                int hi = min(64, p.s_k - kv0);
                 if (p.causal) hi = min(hi, row + p.causal_offset - kv0 + 1);
                 int lo = 0;
                 if (p.window_left >= 0) lo = row + p.causal_offset - p.window_left - kv0;
-                float pr[128];
+                float pr[64];
                 if (!wait_bar_warp(bar(L::bSFull), steps & 1, wc)) return;
                 ptx::tc_fence_after();
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 2; ++q) {
                     uint32_t sr[32];
                     ptx::tmem_ld32(s_tm + q * 32, sr);
                     ptx::tmem_wait_ld();
@@ -428,18 +437,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bar(L::bSFree));
 #pragma unroll
-                for (int k = 0; k < 128; ++k) {
+                for (int k = 0; k < 64; ++k) {
                     const float x = ptx::ex2(fmaf(pr[k], c2, -Lr));
                     pr[k] = (k >= lo && k < hi) ? x : 0.f;
                 }
-                // dS = P (dP - D) -> BF16, into the dS tile (K-major,
-                // 128-byte swizzle: chunk cc of row r at
-                // (r / 8) * 1024 + (r % 8) * 128 + (cc / 8) * 16 KiB + ((cc % 8) ^ (r % 8)) * 16).
+                // dS = P (dP - D) -> BF16, into this warpgroup's half of the
+                // dS tile (K-major, 128-byte swizzle).
                 if (!wait_bar_warp(bar(L::bPFull), steps & 1, wc)) return;
                 if (steps > 0 && !wait_bar_warp(bar(L::bDsFree), (steps - 1) & 1, wc)) return;
                 ptx::tc_fence_after();
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
+                for (int q = 0; q < 2; ++q) {
                     uint32_t dr[32];
                     ptx::tmem_ld32(dp_tm + q * 32, dr);
                     ptx::tmem_wait_ld();
@@ -452,9 +460,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
 #pragma unroll
                     for (int k = 0; k < 4; ++k) {
-                        const int cc = 4 * q + k;
-                        ptx::st_shared_v4(ds_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ xr) << 4),
-                                          w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                        const int cc = 4 * q + k;  // chunk within this half
+                        ptx::st_shared_v4(ds_row + ((cc ^ xr) << 4), w[4 * k], w[4 * k + 1],
+                                          w[4 * k + 2], w[4 * k + 3]);
                     }
                 }
                 ptx::tc_fence_before();
@@ -465,12 +473,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ptx::mbar_arrive(bar(L::bDsFull));
                 }
             }
-            // Epilogue: dQ * scale -> BF16 rows, staged in the dS tile (free
-            // once the last dQ MMA has completed) and stored with TMA.
+            // Epilogue: dQ * scale -> BF16 rows, each warpgroup its 64
+            // columns, staged in its half of the dS tile (free once the last
+            // dQ MMA has completed) and stored with TMA.
             if (!wait_bar_warp(bar(L::bDqFull), items & 1, wc)) return;
             ptx::tc_fence_after();
 #pragma unroll
-            for (int q = 0; q < 4; ++q) {
+            for (int q = 0; q < 2; ++q) {
                 uint32_t v[32];
                 ptx::tmem_ld32(dq_tm + q * 32, v);
                 ptx::tmem_wait_ld();
@@ -482,8 +491,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int cc = 4 * q + k;
-                    ptx::st_shared_v4(ds_row + (cc >> 3) * kHalfTileBytes + (((cc & 7) ^ xr) << 4),
-                                      w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+                    ptx::st_shared_v4(ds_row + ((cc ^ xr) << 4), w[4 * k], w[4 * k + 1],
+                                      w[4 * k + 2], w[4 * k + 3]);
                 }
             }
             ptx::tc_fence_before();
@@ -493,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::mbar_arrive(bar(L::bDqFree));
                 ptx::mbar_arrive(bar(L::bStaged));
             }
-            if (r == 0) {
+            if (warp == 0 && lane == 0) {
                 if (!wait_bar(bar(L::bStaged), items & 1, wc)) return;
                 ptx::tma_store_4d(&tm_dq, sbase + L::kDS, 0, c.h, c.qb * kBlockM, c.b);
                 ptx::tma_store_4d(&tm_dq, sbase + L::kDS + kHalfTileBytes, 64, c.h,
@@ -507,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!wait_bar_warp(bar(L::bStored), items & 1, wc)) return;
             ++items;
         }
-        if (r == 0) ptx::bulk_wait_group0();
+        if (warp == 0 && lane == 0) ptx::bulk_wait_group0();
     }
 
     ptx::tc_fence_before();
