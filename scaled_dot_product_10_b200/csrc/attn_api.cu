@@ -510,9 +510,9 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
         !aligned(workspace, 256))
         return ATTN_ERR_ALIGN;
     if (workspace_bytes < attn_bwd_workspace_bytes(batch, h_q, s_q)) return ATTN_ERR_INVALID;
-    const long long n_qb64 = (s_q + bwd::kBlockQ - 1) / bwd::kBlockQ;
+    const long long n_qb = (s_q + kBlockM - 1) / kBlockM;
     const long long n_kb = (s_k + kBlockN - 1) / kBlockN;
-    if (static_cast<long long>(batch) * h_q * n_qb64 > 0x7fffffffLL ||
+    if (static_cast<long long>(batch) * h_q * n_qb > 0x7fffffffLL ||
         static_cast<long long>(batch) * h_kv * n_kb > 0x7fffffffLL)
         return ATTN_ERR_INVALID;
     int dev = 0;
@@ -529,9 +529,8 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     p.s_q = s_q;
     p.s_k = s_k;
     p.group = h_q / h_kv;
-    p.n_qb = (s_q + kBlockM - 1) / kBlockM;
+    p.n_qb = static_cast<int>(n_qb);
     p.n_kb = static_cast<int>(n_kb);
-    p.n_qb64 = static_cast<int>(n_qb64);
     p.s_q_pad = p.n_qb * kBlockM;
     p.causal = causal;
     p.causal_offset = s_k - s_q;
@@ -544,6 +543,8 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     float* Dw = Lw + static_cast<size_t>(batch) * h_q * p.s_q_pad;
     p.L = Lw;
     p.D = Dw;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
     p.timeout_ns = g_timeout_ns;
     p.status = st->status;
 
@@ -557,12 +558,10 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     bwd::attn_bwd_prep_kernel<<<static_cast<unsigned>(blocks), bwd::kPrepThreads, 0, cs>>>(a);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
-    CUtensorMap tq, tk, tv, tdo, tdq, tq64, tdo64, tdk, tdv;
+    CUtensorMap tq, tk, tv, tdo, tdq;
     if (!encode_map(&tq, q, h_q, s_q, batch) || !encode_map(&tk, k, h_kv, s_k, batch) ||
         !encode_map(&tv, v, h_kv, s_k, batch) || !encode_map(&tdo, dout, h_q, s_q, batch) ||
-        !encode_map(&tdq, dq, h_q, s_q, batch) || !encode_map(&tq64, q, h_q, s_q, batch, 64) ||
-        !encode_map(&tdo64, dout, h_q, s_q, batch, 64) ||
-        !encode_map(&tdk, dk, h_kv, s_k, batch) || !encode_map(&tdv, dv, h_kv, s_k, batch))
+        !encode_map(&tdq, dq, h_q, s_q, batch))
         return ATTN_ERR_CUDA;
 
     // Sections of 4 heads keep the streamed tiles of the heads in flight in
@@ -577,7 +576,7 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     if (p.section > batch * h_kv) p.section = batch * h_kv;
     int grid = p.num_items < st->num_sms ? p.num_items : st->num_sms;
     bwd::dkdv::attn_bwd_dkdv_kernel<<<grid, bwd::dkdv::kThreads, bwd::dkdv::Smem::kAlloc, cs>>>(
-        tq64, tk, tv, tdo64, tdk, tdv, p);
+        tq, tk, tv, tdo, p);
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
 
     // 3. dQ: one item per (query block, batch, query head).

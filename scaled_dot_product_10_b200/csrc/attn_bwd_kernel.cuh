@@ -22,16 +22,18 @@
 //                            keys, thread = row), dQ += dS K on the tensor
 //                            core;
 //   attn_bwd_dkdv_kernel  -- one CTA item per 128-key block of a key/value
-//                            head: K and V stay in shared memory, 64-row
-//                            Q/dO tiles of every query head of the group
-//                            stream through a three-slot ring; S^T = K Q^T
-//                            and dP^T = V dO^T on the tensor core, P^T and
-//                            dS^T by one of two warpgroups (alternate steps,
-//                            thread = key), dV += P^T dO and dK += dS^T Q.
-// In the dK/dV kernel one warpgroup's exponentials run while the other's
-// products are on the tensor core.  (The same split for dQ, with 64-key
-// steps, measured slower on B200 than this single-warpgroup dQ kernel with
-// 128-key steps, which already overlaps S(j+1) with block j's softmax.)
+//                            head: K and V stay in shared memory, 128-row
+//                            Q / dO tiles of every query head of the group
+//                            stream through two-slot rings; S^T = K Q^T and
+//                            dP^T = V dO^T on the tensor core (TMEM), P^T
+//                            and dS^T by two warpgroups (each 64 of the
+//                            step's queries, thread = key), written back to
+//                            TMEM in BF16 over the columns they came from;
+//                            dV += P^T dO and dK += dS^T Q read them there
+//                            as the A operand.
+// Both main kernels issue only N = 128 products: on B200 a 128 x 64 x 16
+// tcgen05.mma takes 55 cycles against 64 for 128 x 128 x 16, so 64-wide
+// steps run the tensor core at about half rate.
 // Splitting dQ from dK/dV costs a second Q K^T and dO V^T but needs no
 // atomics: every output element is written once, by one CTA, and the result
 // is bit-for-bit reproducible.
@@ -42,16 +44,11 @@
 namespace sdpa10 {
 namespace bwd {
 
-constexpr int kBlockQ = 64;             // query rows per dK/dV step
-constexpr int kQTile64Bytes = kBlockQ * kHeadDim * 2;  // 16 KiB: 64 rows x 128
-constexpr int kHalf64Bytes = kQTile64Bytes / 2;         // one 64-column half
-
 struct BwdParams {
     int batch, h_q, h_kv, s_q, s_k;
     int group;             // h_q / h_kv
     int n_qb;              // ceil(s_q / 128)   (dQ kernel)
     int n_kb;              // ceil(s_k / 128)
-    int n_qb64;            // ceil(s_q / 64)    (dK/dV kernel)
     int s_q_pad;           // row stride of the L / D workspace: n_qb * 128
     int causal;
     int causal_offset;     // s_k - s_q
@@ -71,6 +68,8 @@ struct BwdParams {
     float scale_log2;      // scale * log2(e)
     const float* L;        // [batch][h_q][s_q_pad]  LSE * log2(e) (+inf padding)
     const float* D;        // [batch][h_q][s_q_pad]  rowsum(dO * O) (0 padding)
+    __nv_bfloat16* dk;     // [batch][s_k][h_kv][128] outputs of the dK/dV kernel
+    __nv_bfloat16* dv;
     unsigned long long timeout_ns;
     unsigned int* status;
 };
@@ -535,33 +534,28 @@ namespace sdpa10 {
 namespace bwd {
 namespace dkdv {
 
-// Two compute warpgroups take alternate 64-row steps (warps 0-3 the even
-// global steps, warps 4-7 the odd ones), so one warpgroup's exponentials and
-// dS^T run while the other's tiles are on the tensor core; warp 8 is the
-// TMA producer and warp 9 the MMA issuer.
+// Two compute warpgroups split every 128-query step by columns: warpgroup w
+// takes queries 64w .. 64w + 63 of the step for all 128 keys of the block
+// (thread = key = TMEM lane).  Warp 8 is the TMA producer, warp 9 the MMA
+// issuer.
 constexpr int kThreads = 320;
 constexpr int kLoadWarp = 8;
 constexpr int kMmaWarp = 9;
-constexpr int kQDStages = 3;
+constexpr int kStages = 2;  // slots of the Q ring and of the dO ring
 
 struct Smem {
-    static constexpr int kK = 0;                              // K tile (A of S^T = K Q^T)
-    static constexpr int kV = kTileBytes;                     // V tile (A of dP^T = V dO^T)
-    static constexpr int kQD = 2 * kTileBytes;                // ring of 3 x (Q 64 rows, dO 64 rows)
-    static constexpr int kQDSlot = 2 * kQTile64Bytes;         // 32 KiB per slot
-    // Per warpgroup w: P^T_w then dS^T_w ([128 keys x 64], 16 KiB each),
-    // 32 KiB contiguous; at the end of an item warpgroup 0 stages dV and
-    // warpgroup 1 stages dK there for the TMA store.
-    static constexpr int kWG = kQD + kQDStages * kQDSlot;
-    static constexpr int kWGBytes = 2 * kQTile64Bytes;
-    static constexpr int kLD = kWG + 2 * kWGBytes;            // ring of 3 x (L[64], D[64])
-    static constexpr int kBars = kLD + kQDStages * 512;
-    static constexpr int bKVFull = 0, bKVEmpty = 1, bQDFull = 2, bQDEmpty = 2 + kQDStages,
-                         bSFull = 2 + 2 * kQDStages,       // [2] per warpgroup from here on
-                         bSFree = bSFull + 2, bPFull = bSFree + 2, bPFree = bPFull + 2,
-                         bPTFull = bPFree + 2, bPTFree = bPTFull + 2, bDSTFull = bPTFree + 2,
-                         bDSTFree = bDSTFull + 2, bStaged = bDSTFree + 2, bStored = bStaged + 2,
-                         bAccFull = bStored + 2, bAccFree = bAccFull + 1, bDrain = bAccFree + 1,
+    static constexpr int kK = 0;                             // K tile (A of S^T = K Q^T)
+    static constexpr int kV = kTileBytes;                    // V tile (A of dP^T = V dO^T)
+    static constexpr int kQ = 2 * kTileBytes;                // ring of Q tiles (128 rows)
+    static constexpr int kDO = kQ + kStages * kTileBytes;    // ring of dO tiles
+    static constexpr int kLD = kDO + kStages * kTileBytes;   // per Q slot: L[128], D[128]
+    static constexpr int kLDSlot = 2 * kBlockM * 4;
+    static constexpr int kBars = kLD + kStages * kLDSlot;
+    static constexpr int bKFull = 0, bKEmpty = 1, bVFull = 2, bVEmpty = 3, bQFull = 4,
+                         bQEmpty = bQFull + kStages, bOFull = bQEmpty + kStages,
+                         bOEmpty = bOFull + kStages, bSFull = bOEmpty + kStages,
+                         bPFull = bSFull + 1, bPTFull = bPFull + 1, bDSTFull = bPTFull + 1,
+                         bAccFull = bDSTFull + 1, bAccFree = bAccFull + 1, bDrain = bAccFree + 1,
                          kNumBars = bDrain + 1;
     static constexpr int kTmemSlot = kBars + kNumBars * 8;
     static constexpr int kAbort = kTmemSlot + 4;
@@ -570,10 +564,15 @@ struct Smem {
 };
 static_assert(Smem::kAlloc <= 232448, "dK/dV shared memory exceeds the per-CTA limit");
 
+// TMEM columns: S^T at 0 (P^T in BF16 over its first half of each
+// warpgroup's 64 columns), dP^T at 128 (dS^T likewise), dV at 256, dK at 384.
+constexpr uint32_t kTmS = 0, kTmDP = 128, kTmDV = 256, kTmDK = 384;
+
 // Item t -> (key block, batch, key/value head): by section of heads, then
 // key block ascending (under the causal mask the first key blocks are seen
-// by the most query rows: longest first), then head.  The item walks the query heads of
-// the group and, for each, the 64-row query blocks that see the key block.
+// by the most query rows: longest first), then head.  The item walks the
+// query heads of the group and, for each, the 128-row query blocks that see
+// the key block.
 struct Cursor {
     int round, t;
     int b, g, kb;
@@ -588,17 +587,17 @@ struct Cursor {
         const int bg = sec * p.section + (r - kb * in_sec);
         b = p.div_h_kv.div(bg);
         g = bg - b * p.h_kv;
-        int lo = 0, hi = p.n_qb64;
+        int lo = 0, hi = p.n_qb;
         if (p.causal) {
             // Query i sees key 128 kb (the block's first key) iff
-            // i >= 128 kb - causal_offset: floor division by 64.
-            lo = max(0, (kb * kBlockN - p.causal_offset) >> 6);
+            // i >= 128 kb - causal_offset: floor division by 128.
+            lo = max(0, (kb * kBlockN - p.causal_offset) >> 7);
         }
         if (p.window_left >= 0) {
             // Query i still sees the block's last key iff
             // i <= 128 kb + 127 + window_left - causal_offset.
             const int last = kb * kBlockN + kBlockN - 1 + p.window_left - p.causal_offset;
-            hi = min(hi, (last >> 6) + 1);
+            hi = min(hi, (last >> 7) + 1);
         }
         qlo = lo;
         nq = max(0, hi - lo);
@@ -616,15 +615,19 @@ struct Cursor {
     __device__ __forceinline__ void next(const BwdParams& p) { ++round; settle(p); }
     __device__ __forceinline__ bool valid(const BwdParams& p) const { return t < p.num_items; }
     __device__ __forceinline__ int steps(const BwdParams& p) const { return p.group * nq; }
+    // Query head and query block of step s.
+    __device__ __forceinline__ void step(const BwdParams& p, int s, int& h, int& qb) const {
+        const int hl = s / nq;
+        qb = qlo + (s - hl * nq);
+        h = g * p.group + hl;
+    }
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q64,
+    attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
                          const __grid_constant__ CUtensorMap tm_v,
-                         const __grid_constant__ CUtensorMap tm_do64,
-                         const __grid_constant__ CUtensorMap tm_dk,
-                         const __grid_constant__ CUtensorMap tm_dv,
+                         const __grid_constant__ CUtensorMap tm_do,
                          const __grid_constant__ BwdParams p) {
     using L = Smem;
     extern __shared__ uint8_t smem_raw[];
@@ -638,37 +641,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
     if (threadIdx.x == 0) {
-        ptx::mbar_init(bar(L::bKVFull), 1);
-        ptx::mbar_init(bar(L::bKVEmpty), 1);
-        for (int i = 0; i < kQDStages; ++i) {
-            ptx::mbar_init(bar(L::bQDFull + i), 1);
-            ptx::mbar_init(bar(L::bQDEmpty + i), 1);
+        ptx::mbar_init(bar(L::bKFull), 1);
+        ptx::mbar_init(bar(L::bKEmpty), 1);
+        ptx::mbar_init(bar(L::bVFull), 1);
+        ptx::mbar_init(bar(L::bVEmpty), 1);
+        for (int i = 0; i < kStages; ++i) {
+            ptx::mbar_init(bar(L::bQFull + i), 1);
+            ptx::mbar_init(bar(L::bQEmpty + i), 1);
+            ptx::mbar_init(bar(L::bOFull + i), 1);
+            ptx::mbar_init(bar(L::bOEmpty + i), 1);
         }
-        for (int w = 0; w < 2; ++w) {
-            ptx::mbar_init(bar(L::bSFull + w), 1);
-            ptx::mbar_init(bar(L::bSFree + w), 4);
-            ptx::mbar_init(bar(L::bPFull + w), 1);
-            ptx::mbar_init(bar(L::bPFree + w), 4);
-            ptx::mbar_init(bar(L::bPTFull + w), 4);
-            ptx::mbar_init(bar(L::bPTFree + w), 1);
-            ptx::mbar_init(bar(L::bDSTFull + w), 4);
-            ptx::mbar_init(bar(L::bDSTFree + w), 1);
-            ptx::mbar_init(bar(L::bStaged + w), 4);
-            ptx::mbar_init(bar(L::bStored + w), 1);
-        }
+        ptx::mbar_init(bar(L::bSFull), 1);
+        ptx::mbar_init(bar(L::bPFull), 1);
+        ptx::mbar_init(bar(L::bPTFull), 8);   // every compute warp has written P^T
+        ptx::mbar_init(bar(L::bDSTFull), 8);  // ... dS^T
         ptx::mbar_init(bar(L::bAccFull), 1);
-        ptx::mbar_init(bar(L::bAccFree), 8);  // both warpgroups have read dV / dK
+        ptx::mbar_init(bar(L::bAccFree), 8);  // every compute warp has read dV / dK
         ptx::mbar_init(bar(L::bDrain), 1);
         *abort_flag = 0;
         ptx::fence_mbar_init();
     }
     if (warp == kLoadWarp && lane == 0) {
-        ptx::prefetch_tmap(&tm_q64);
+        ptx::prefetch_tmap(&tm_q);
         ptx::prefetch_tmap(&tm_k);
         ptx::prefetch_tmap(&tm_v);
-        ptx::prefetch_tmap(&tm_do64);
-        ptx::prefetch_tmap(&tm_dk);
-        ptx::prefetch_tmap(&tm_dv);
+        ptx::prefetch_tmap(&tm_do);
     }
     if (warp == kMmaWarp) {
         ptx::tmem_alloc(ptx::smem_u32(tmem_slot), kTmemCols);
@@ -677,146 +674,187 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    // TMEM: S^T_0 | S^T_1 | dP^T_0 | dP^T_1 (64 columns each) | dV | dK at
-    // columns 0, 64, 128, 192, 256, 384.
     const uint32_t tmem = *tmem_slot;
     const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
-    auto qd_addr = [&](uint32_t u) { return sbase + L::kQD + (u % kQDStages) * L::kQDSlot; };
+    auto q_addr = [&](uint32_t u) { return sbase + L::kQ + (u % kStages) * kTileBytes; };
+    auto do_addr = [&](uint32_t u) { return sbase + L::kDO + (u % kStages) * kTileBytes; };
 
     if (warp == kLoadWarp) {
         // ============================================================ producer
+        // Per item: K, Q of its first step, V, dO of its first step, then Q
+        // and dO of the following steps; K (V) of the next item is loaded as
+        // soon as the last S^T (dP^T) of this one has been read.
         if (lane == 0) {
             const uint64_t pol_kv = ptx::policy_evict_first();
             const uint64_t pol_q = ptx::policy_evict_last();
-            uint32_t kv_loads = 0, qd_loads = 0;
+            uint32_t items = 0, loads = 0;
             bool ok = true;
+            auto load_q = [&](const Cursor& c, int s) -> bool {
+                int h, qb;
+                c.step(p, s, h, qb);
+                const uint32_t slot = loads % kStages;
+                if (!wait_bar(bar(L::bQEmpty + slot), ((loads / kStages) & 1) ^ 1, wc)) return false;
+                const uint32_t full = bar(L::bQFull + slot);
+                ptx::mbar_arrive_expect_tx(full, kTileBytes + L::kLDSlot);
+#pragma unroll
+                for (int half = 0; half < 2; ++half)
+                    ptx::tma_load_4d(q_addr(loads) + half * kHalfTileBytes, &tm_q, full, 64 * half,
+                                     h, qb * kBlockM, c.b, pol_q);
+                const size_t stat =
+                    (static_cast<size_t>(c.b) * p.h_q + h) * p.s_q_pad + qb * kBlockM;
+                const uint32_t ld = sbase + L::kLD + slot * L::kLDSlot;
+                ptx::bulk_load(ld, p.L + stat, kBlockM * 4, full);
+                ptx::bulk_load(ld + kBlockM * 4, p.D + stat, kBlockM * 4, full);
+                return true;
+            };
+            auto load_do = [&](const Cursor& c, int s) -> bool {
+                int h, qb;
+                c.step(p, s, h, qb);
+                const uint32_t slot = loads % kStages;
+                if (!wait_bar(bar(L::bOEmpty + slot), ((loads / kStages) & 1) ^ 1, wc)) return false;
+                const uint32_t full = bar(L::bOFull + slot);
+                ptx::mbar_arrive_expect_tx(full, kTileBytes);
+#pragma unroll
+                for (int half = 0; half < 2; ++half)
+                    ptx::tma_load_4d(do_addr(loads) + half * kHalfTileBytes, &tm_do, full,
+                                     64 * half, h, qb * kBlockM, c.b, pol_q);
+                return true;
+            };
             Cursor c;
             for (c.start(p); ok && c.valid(p); c.next(p)) {
-                if (!(ok = wait_bar(bar(L::bKVEmpty), (kv_loads & 1) ^ 1, wc))) break;
-                ptx::mbar_arrive_expect_tx(bar(L::bKVFull), 2 * kTileBytes);
+                const uint32_t ph = (items & 1) ^ 1;
+                if (!(ok = wait_bar(bar(L::bKEmpty), ph, wc))) break;
+                ptx::mbar_arrive_expect_tx(bar(L::bKFull), kTileBytes);
 #pragma unroll
-                for (int half = 0; half < 2; ++half) {
-                    ptx::tma_load_4d(sbase + L::kK + half * kHalfTileBytes, &tm_k, bar(L::bKVFull),
+                for (int half = 0; half < 2; ++half)
+                    ptx::tma_load_4d(sbase + L::kK + half * kHalfTileBytes, &tm_k, bar(L::bKFull),
                                      64 * half, c.g, c.kb * kBlockN, c.b, pol_kv);
-                    ptx::tma_load_4d(sbase + L::kV + half * kHalfTileBytes, &tm_v, bar(L::bKVFull),
+                if (!(ok = load_q(c, 0))) break;
+                if (!(ok = wait_bar(bar(L::bVEmpty), ph, wc))) break;
+                ptx::mbar_arrive_expect_tx(bar(L::bVFull), kTileBytes);
+#pragma unroll
+                for (int half = 0; half < 2; ++half)
+                    ptx::tma_load_4d(sbase + L::kV + half * kHalfTileBytes, &tm_v, bar(L::bVFull),
                                      64 * half, c.g, c.kb * kBlockN, c.b, pol_kv);
-                }
-                ++kv_loads;
+                if (!(ok = load_do(c, 0))) break;
+                ++loads;
+                ++items;
                 const int n = c.steps(p);
-                for (int s = 0; s < n && ok; ++s) {
-                    const int hl = s / c.nq;
-                    const int qb = c.qlo + (s - hl * c.nq);
-                    const int h = c.g * p.group + hl;
-                    const uint32_t slot = qd_loads % kQDStages;
-                    if (!(ok = wait_bar(bar(L::bQDEmpty + slot),
-                                        ((qd_loads / kQDStages) & 1) ^ 1, wc)))
-                        break;
-                    const uint32_t full = bar(L::bQDFull + slot);
-                    const uint32_t dst = qd_addr(qd_loads);
-                    ptx::mbar_arrive_expect_tx(full, 2 * kQTile64Bytes + 512);
-#pragma unroll
-                    for (int half = 0; half < 2; ++half) {
-                        ptx::tma_load_4d(dst + half * kHalf64Bytes, &tm_q64, full, 64 * half, h,
-                                         qb * kBlockQ, c.b, pol_q);
-                        ptx::tma_load_4d(dst + kQTile64Bytes + half * kHalf64Bytes, &tm_do64, full,
-                                         64 * half, h, qb * kBlockQ, c.b, pol_q);
-                    }
-                    const size_t stat =
-                        (static_cast<size_t>(c.b) * p.h_q + h) * p.s_q_pad + qb * kBlockQ;
-                    ptx::bulk_load(sbase + L::kLD + slot * 512, p.L + stat, 256, full);
-                    ptx::bulk_load(sbase + L::kLD + slot * 512 + 256, p.D + stat, 256, full);
-                    ++qd_loads;
+                for (int s = 1; s < n && ok; ++s) {
+                    if (!(ok = load_q(c, s))) break;
+                    if (!(ok = load_do(c, s))) break;
+                    ++loads;
                 }
             }
-            if (kv_loads > 0) wait_slow(bar(L::bKVFull), (kv_loads - 1) & 1, wc, false);
-            for (int i = 0; i < kQDStages && i < static_cast<int>(qd_loads); ++i) {
-                const uint32_t f = qd_loads - 1 - i;
-                wait_slow(bar(L::bQDFull + f % kQDStages), (f / kQDStages) & 1, wc, false);
+            // Let every issued copy land before the CTA can exit.
+            if (items > 0) {
+                wait_slow(bar(L::bKFull), (items - 1) & 1, wc, false);
+                wait_slow(bar(L::bVFull), (items - 1) & 1, wc, false);
+            }
+            for (int i = 0; i < kStages && i < static_cast<int>(loads); ++i) {
+                const uint32_t f = loads - 1 - i;
+                wait_slow(bar(L::bQFull + f % kStages), (f / kStages) & 1, wc, false);
+                wait_slow(bar(L::bOFull + f % kStages), (f / kStages) & 1, wc, false);
             }
         }
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
         if (lane == 0) {
-            constexpr uint32_t kIdS = idesc_bf16_f32(kBlockN, kBlockQ, 0, 0);   // K Q^T, V dO^T
+            constexpr uint32_t kIdS = idesc_bf16_f32(kBlockN, kBlockM, 0, 0);     // K Q^T, V dO^T
             constexpr uint32_t kIdAcc = idesc_bf16_f32(kBlockN, kHeadDim, 0, 1);  // P^T dO, dS^T Q
             const uint32_t k_lo = desc_lo_sw128(sbase + L::kK, 16);
             const uint32_t v_lo = desc_lo_sw128(sbase + L::kV, 16);
-            const uint32_t dv_tm = tmem + 256, dk_tm = tmem + 384;
-            uint32_t items = 0, gs0 = 0;
-            bool ok = true;
-            // X^T = A B^T with A a [128 x 128] K-major tile (K or V) and B a
-            // 64-row K-major tile (Q or dO): 8 K-steps; the 64-row tile's
-            // second 64-column half is 8 KiB on.
-            auto gemm_t = [&](uint32_t d_tm, uint32_t a_lo, uint32_t b_lo) {
+            // X^T = A B^T with A the [128 x 128] K or V tile and B the
+            // 128-row Q or dO tile, both K-major: 8 K-steps of 16.
+            auto gemm_t = [&](uint32_t d_tm, uint32_t a_lo, uint32_t b_addr) {
+                const uint32_t b_lo = desc_lo_sw128(b_addr, 16);
 #pragma unroll
                 for (int k = 0; k < kHeadDim / 16; ++k) {
-                    const uint32_t oa = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
-                    const uint32_t ob = ((k >> 2) * kHalf64Bytes + (k & 3) * 32) >> 4;
-                    ptx::mma_ss(d_tm, desc_from_lo(a_lo + oa), desc_from_lo(b_lo + ob), kIdS,
+                    const uint32_t o = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
+                    ptx::mma_ss(d_tm, desc_from_lo(a_lo + o), desc_from_lo(b_lo + o), kIdS,
                                 k > 0 ? 1u : 0u);
                 }
             };
-            // Acc += A B with A a [128 x 64] K-major tile (P^T or dS^T, one
-            // 64-column half) and B the 64-row tile read MN-major (head dim
-            // contiguous, halves 8 KiB apart): 4 K-steps of 16 rows = 2 KiB.
-            auto gemm_acc = [&](uint32_t d_tm, uint32_t a_lo, uint32_t b_addr, bool acc) {
-                const uint32_t b_lo = desc_lo_sw128(b_addr, kHalf64Bytes);
+            // Acc += A B with A = P^T or dS^T [128 keys x 128 queries] in
+            // TMEM (queries 0-63 packed in the columns at a_tm, queries
+            // 64-127 at a_tm + 64) and B the 128-row Q or dO tile read
+            // MN-major: 16 queries = 2 KiB per K-step, head-dim halves 16 KiB
+            // apart.
+            auto gemm_acc = [&](uint32_t d_tm, uint32_t a_tm, uint32_t b_addr, bool acc) {
+                const uint32_t b_lo = desc_lo_sw128(b_addr, kHalfTileBytes);
 #pragma unroll
-                for (int k = 0; k < kBlockQ / 16; ++k)
-                    ptx::mma_ss(d_tm, desc_from_lo(a_lo + ((k * 32) >> 4)),
+                for (int k = 0; k < kBlockM / 16; ++k)
+                    ptx::mma_ts(d_tm, a_tm + (k >> 2) * 64 + (k & 3) * 8,
                                 desc_from_lo(b_lo + ((k * 2048) >> 4)), kIdAcc,
                                 (acc || k > 0) ? 1u : 0u);
             };
-            // S^T and dP^T of global step gs into warpgroup (gs & 1)'s
-            // columns once that warpgroup has read its previous ones.
-            auto scores = [&](uint32_t gs) -> bool {
-                const uint32_t w = gs & 1, i = gs >> 1;
-                if (!wait_bar(bar(L::bQDFull + gs % kQDStages), (gs / kQDStages) & 1, wc))
-                    return false;
-                if (i > 0 && !wait_bar(bar(L::bSFree + w), (i - 1) & 1, wc)) return false;
+            uint32_t gs = 0, items = 0, kv = 0;
+            bool ok = true;
+            Cursor c;
+            c.start(p);
+            // S^T(gs) once K and Q are in; dP^T(gs) once V and dO are in.  A
+            // new item's first S^T / dP^T also waits for its K / V; the last
+            // S^T / dP^T of an item releases K / V for the next one.
+            auto issue_s = [&](uint32_t u, bool first, bool last) -> bool {
+                if (first && !wait_bar(bar(L::bKFull), kv & 1, wc)) return false;
+                if (!wait_bar(bar(L::bQFull + u % kStages), (u / kStages) & 1, wc)) return false;
                 ptx::tc_fence_after();
-                gemm_t(tmem + 64 * w, k_lo, desc_lo_sw128(qd_addr(gs), 16));
-                ptx::mma_commit(bar(L::bSFull + w));
-                if (i > 0 && !wait_bar(bar(L::bPFree + w), (i - 1) & 1, wc)) return false;
-                ptx::tc_fence_after();
-                gemm_t(tmem + 128 + 64 * w, v_lo, desc_lo_sw128(qd_addr(gs) + kQTile64Bytes, 16));
-                ptx::mma_commit(bar(L::bPFull + w));
+                gemm_t(tmem + kTmS, k_lo, q_addr(u));
+                ptx::mma_commit(bar(L::bSFull));
+                if (last) ptx::mma_commit(bar(L::bKEmpty));
                 return true;
             };
-            Cursor c;
-            for (c.start(p); ok && c.valid(p); c.next(p)) {
-                const int n = c.steps(p);
-                if (!(ok = wait_bar(bar(L::bKVFull), items & 1, wc))) break;
-                // Per item: S^T, dP^T of its first two steps, then per step
-                // s: dV(s), dK(s), then S^T, dP^T of step s + 2 (same
-                // warpgroup) -- the other warpgroup's step s + 1 runs on the
-                // tensor core while this one's exponentials run.
-                if (!(ok = scores(gs0))) break;
-                if (n > 1 && !(ok = scores(gs0 + 1))) break;
-                // dV / dK of the previous item must have been read out.
-                if (items > 0 && !(ok = wait_bar(bar(L::bAccFree), (items - 1) & 1, wc))) break;
-                ++items;
-                for (int s = 0; s < n && ok; ++s) {
-                    const uint32_t gs = gs0 + s, w = gs & 1, i = gs >> 1;
-                    const uint32_t pt_lo = desc_lo_sw128(sbase + L::kWG + w * L::kWGBytes, 16);
-                    const uint32_t dst_lo =
-                        desc_lo_sw128(sbase + L::kWG + w * L::kWGBytes + kQTile64Bytes, 16);
-                    if (!(ok = wait_bar(bar(L::bPTFull + w), i & 1, wc))) break;
+            auto issue_dp = [&](uint32_t u, bool first, bool last) -> bool {
+                if (first && !wait_bar(bar(L::bVFull), kv & 1, wc)) return false;
+                if (!wait_bar(bar(L::bOFull + u % kStages), (u / kStages) & 1, wc)) return false;
+                ptx::tc_fence_after();
+                gemm_t(tmem + kTmDP, v_lo, do_addr(u));
+                ptx::mma_commit(bar(L::bPFull));
+                if (last) ptx::mma_commit(bar(L::bVEmpty));
+                return true;
+            };
+            if (c.valid(p)) {
+                int n = c.steps(p), s = 0;
+                ok = issue_s(0, true, n == 1) && issue_dp(0, true, n == 1);
+                ++kv;
+                while (ok) {
+                    // Step gs (step s of n of the current item).  P^T(gs) in
+                    // TMEM over S^T: dV += P^T dO.
+                    if (!(ok = wait_bar(bar(L::bPTFull), gs & 1, wc))) break;
+                    if (s == 0 && items > 0 && !(ok = wait_bar(bar(L::bAccFree), (items - 1) & 1, wc)))
+                        break;
                     ptx::tc_fence_after();
-                    gemm_acc(dv_tm, pt_lo, qd_addr(gs) + kQTile64Bytes, s > 0);
-                    ptx::mma_commit(bar(L::bPTFree + w));
-                    if (!(ok = wait_bar(bar(L::bDSTFull + w), i & 1, wc))) break;
+                    gemm_acc(tmem + kTmDV, tmem + kTmS, do_addr(gs), s > 0);
+                    ptx::mma_commit(bar(L::bOEmpty + gs % kStages));
+                    // The next step's S^T overwrites P^T(gs) only after the
+                    // dV products above (the tensor core runs in issue order).
+                    Cursor cn = c;
+                    int sn = s + 1, nn = n;
+                    if (sn == n) {
+                        cn.next(p);
+                        sn = 0;
+                        nn = cn.valid(p) ? cn.steps(p) : 0;
+                    }
+                    const bool more = cn.valid(p);
+                    if (more && !(ok = issue_s(gs + 1, sn == 0, sn == nn - 1))) break;
+                    // dS^T(gs) in TMEM over dP^T: dK += dS^T Q.
+                    if (!(ok = wait_bar(bar(L::bDSTFull), gs & 1, wc))) break;
                     ptx::tc_fence_after();
-                    gemm_acc(dk_tm, dst_lo, qd_addr(gs), s > 0);
-                    ptx::mma_commit(bar(L::bDSTFree + w));
-                    ptx::mma_commit(bar(L::bQDEmpty + gs % kQDStages));
-                    if (s + 2 < n && !(ok = scores(gs + 2))) break;
+                    gemm_acc(tmem + kTmDK, tmem + kTmDP, q_addr(gs), s > 0);
+                    ptx::mma_commit(bar(L::bQEmpty + gs % kStages));
+                    if (s == n - 1) {
+                        ptx::mma_commit(bar(L::bAccFull));
+                        ++items;
+                    }
+                    if (more && !(ok = issue_dp(gs + 1, sn == 0, sn == nn - 1))) break;
+                    if (!more) break;
+                    if (sn == 0) ++kv;
+                    c = cn;
+                    s = sn;
+                    n = nn;
+                    ++gs;
                 }
-                if (!ok) break;
-                gs0 += n;
-                ptx::mma_commit(bar(L::bKVEmpty));
-                ptx::mma_commit(bar(L::bAccFull));
             }
             ptx::mma_commit(bar(L::bDrain));
             wait_slow(bar(L::bDrain), 0, wc, false);
@@ -824,57 +862,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else {
         // ============================================================ compute
-        // Warpgroup w = warp / 4; thread r owns key row r of the block (TMEM
-        // lane r) and takes the global steps gs with gs % 2 == w.
+        // Warpgroup w = warp / 4 takes query columns 64w .. 64w + 63 of each
+        // step; thread r owns key row r of the block (TMEM lane r).
         const int w = warp >> 2;
         const int r = (warp & 3) * 32 + lane;
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-        const uint32_t s_tm = tmem + lane_base + 64 * w, dp_tm = tmem + lane_base + 128 + 64 * w;
-        const uint32_t acc_tm = tmem + lane_base + (w ? 384 : 256);  // dK (w 1) or dV (w 0)
-        // Row r of a [128 x 64] K-major tile: 8 chunks of 16 bytes, chunk cc
-        // at (r / 8) * 1024 + (r % 8) * 128 + ((cc ^ (r % 8)) * 16).
-        const uint32_t xr = static_cast<uint32_t>(r & 7);
-        const uint32_t wg_base = sbase + L::kWG + w * L::kWGBytes;
-        const uint32_t row_off = (r >> 3) * 1024 + (r & 7) * 128;
-        const uint32_t pt_row = wg_base + row_off;
-        const uint32_t dst_row = wg_base + kQTile64Bytes + row_off;
-        const uint32_t st_row = wg_base + row_off;  // [128 x 128] staging, halves 16 KiB apart
+        const uint32_t s_tm = tmem + lane_base + kTmS + 64 * w;
+        const uint32_t dp_tm = tmem + lane_base + kTmDP + 64 * w;
+        const uint32_t acc_tm = tmem + lane_base + (w ? kTmDK : kTmDV);
+        __nv_bfloat16* const out = w ? p.dk : p.dv;
+        const float f = w ? p.scale : 1.f;
         const float c2 = p.scale_log2;
-        uint32_t items = 0, gs0 = 0, mine = 0;  // mine: steps this warpgroup has done
+        uint32_t gs = 0, items = 0;
         Cursor c;
         for (c.start(p); c.valid(p); c.next(p)) {
             const int n = c.steps(p);
             const int key = c.kb * kBlockN + r;
-            for (int s = (gs0 & 1) == static_cast<uint32_t>(w) ? 0 : 1; s < n; s += 2, ++mine) {
-                const uint32_t gs = gs0 + s;
-                const int hl = s / c.nq;
-                const int qb = c.qlo + (s - hl * c.nq);
-                // Visible query columns of this key row: [lo, hi].
-                int lo = 0, hi = kBlockQ - 1;
-                if (p.causal) lo = key - p.causal_offset - qb * kBlockQ;
-                if (p.window_left >= 0)
-                    hi = min(hi, key + p.window_left - p.causal_offset - qb * kBlockQ);
-                const uint32_t slot = gs % kQDStages;
-                const uint32_t sL = sbase + L::kLD + slot * 512;  // L[64], then D[64]
-                const uint32_t sD = sL + 256;
+            for (int s = 0; s < n; ++s, ++gs) {
+                int h, qb;
+                c.step(p, s, h, qb);
+                // Visible columns j (query qb*128 + 64w + j) of this key row:
+                // lo <= j <= hi.
+                const int q0 = qb * kBlockM + 64 * w;
+                int lo = 0, hi = 63;
+                if (p.causal) lo = key - p.causal_offset - q0;
+                if (p.window_left >= 0) hi = min(hi, key + p.window_left - p.causal_offset - q0);
+                const uint32_t slot = gs % kStages;
+                const uint32_t sL = sbase + L::kLD + slot * L::kLDSlot + 4 * 64 * w;
+                const uint32_t sD = sL + kBlockM * 4;
                 float pt[64];
-                // L and D of this step's rows arrive with its Q / dO tiles
-                // (the slot is refilled only after this step's dK MMA, which
-                // waits for this warpgroup).
-                if (!wait_bar_warp(bar(L::bQDFull + slot), (gs / kQDStages) & 1, wc)) return;
-                if (!wait_bar_warp(bar(L::bSFull + w), mine & 1, wc)) return;
+                // L and D arrive with the step's Q tile; that slot is refilled
+                // only after this step's dK products, which wait for dS^T.
+                if (!wait_bar_warp(bar(L::bQFull + slot), (gs / kStages) & 1, wc)) return;
+                if (!wait_bar_warp(bar(L::bSFull), gs & 1, wc)) return;
                 ptx::tc_fence_after();
-#pragma unroll
-                for (int q = 0; q < 2; ++q) {
-                    uint32_t sr[32];
-                    ptx::tmem_ld32(s_tm + q * 32, sr);
+                {
+                    uint32_t s0[32], s1[32];
+                    ptx::tmem_ld32(s_tm, s0);
+                    ptx::tmem_ld32(s_tm + 32, s1);
                     ptx::tmem_wait_ld();
 #pragma unroll
-                    for (int k = 0; k < 32; ++k) pt[q * 32 + k] = __uint_as_float(sr[k]);
+                    for (int k = 0; k < 32; ++k) {
+                        pt[k] = __uint_as_float(s0[k]);
+                        pt[32 + k] = __uint_as_float(s1[k]);
+                    }
                 }
-                ptx::tc_fence_before();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(L::bSFree + w));
 #pragma unroll
                 for (int k4 = 0; k4 < 16; ++k4) {
                     const float4 l4 = ptx::ld_shared_f4(sL + 16 * k4);  // same address: broadcast
@@ -886,22 +918,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pt[k] = (k >= lo && k <= hi) ? x : 0.f;
                     }
                 }
-                // P^T -> BF16 into this warpgroup's tile once its last dV
-                // MMA has read it.
-                if (mine > 0 && !wait_bar_warp(bar(L::bPTFree + w), (mine - 1) & 1, wc)) return;
+                // P^T in BF16 over the first 32 of this warpgroup's S^T
+                // columns (read above by this thread only).
+                {
+                    uint32_t pk[32];
 #pragma unroll
-                for (int cc = 0; cc < 8; ++cc)
-                    ptx::st_shared_v4(pt_row + ((cc ^ xr) << 4),
-                                      ptx::pack_bf16x2(pt[8 * cc], pt[8 * cc + 1]),
-                                      ptx::pack_bf16x2(pt[8 * cc + 2], pt[8 * cc + 3]),
-                                      ptx::pack_bf16x2(pt[8 * cc + 4], pt[8 * cc + 5]),
-                                      ptx::pack_bf16x2(pt[8 * cc + 6], pt[8 * cc + 7]));
-                ptx::fence_proxy_async_smem();
+                    for (int j = 0; j < 32; ++j) pk[j] = ptx::pack_bf16x2(pt[2 * j], pt[2 * j + 1]);
+                    ptx::tmem_st32(s_tm, pk);
+                    ptx::tmem_wait_st();
+                }
+                ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(L::bPTFull + w));
-                // dS^T = P^T (dP^T - D) -> BF16.
-                if (!wait_bar_warp(bar(L::bPFull + w), mine & 1, wc)) return;
-                if (mine > 0 && !wait_bar_warp(bar(L::bDSTFree + w), (mine - 1) & 1, wc)) return;
+                if (lane == 0) ptx::mbar_arrive(bar(L::bPTFull));
+                // dS^T = P^T (dP^T - D), BF16 over the first 32 of this
+                // warpgroup's dP^T columns.
+                if (!wait_bar_warp(bar(L::bPFull), gs & 1, wc)) return;
                 ptx::tc_fence_after();
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
@@ -919,66 +950,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                         }
                     }
                 }
+                {
+                    uint32_t pk[32];
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) pk[j] = ptx::pack_bf16x2(pt[2 * j], pt[2 * j + 1]);
+                    ptx::tmem_st32(dp_tm, pk);
+                    ptx::tmem_wait_st();
+                }
                 ptx::tc_fence_before();
                 __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(L::bPFree + w));
-#pragma unroll
-                for (int cc = 0; cc < 8; ++cc)
-                    ptx::st_shared_v4(dst_row + ((cc ^ xr) << 4),
-                                      ptx::pack_bf16x2(pt[8 * cc], pt[8 * cc + 1]),
-                                      ptx::pack_bf16x2(pt[8 * cc + 2], pt[8 * cc + 3]),
-                                      ptx::pack_bf16x2(pt[8 * cc + 4], pt[8 * cc + 5]),
-                                      ptx::pack_bf16x2(pt[8 * cc + 6], pt[8 * cc + 7]));
-                ptx::fence_proxy_async_smem();
-                __syncwarp();
-                if (lane == 0) ptx::mbar_arrive(bar(L::bDSTFull + w));
+                if (lane == 0) ptx::mbar_arrive(bar(L::bDSTFull));
             }
-            gs0 += n;
-            // Epilogue: warpgroup 0 writes dV, warpgroup 1 dK * scale, as
-            // BF16 rows staged in its own 32 KiB (its P^T and dS^T tiles, free
-            // once every MMA of the item has completed) and stored with TMA
-            // (rows past s_k are clipped by the tensor map).
+            // Epilogue: warpgroup 0 writes dV, warpgroup 1 dK * scale; each
+            // thread stores its key row (256 contiguous bytes) directly.
             if (!wait_bar_warp(bar(L::bAccFull), items & 1, wc)) return;
             ptx::tc_fence_after();
-            const float f = w ? p.scale : 1.f;
+            __nv_bfloat16* row =
+                out + ((static_cast<size_t>(c.b) * p.s_k + key) * p.h_kv + c.g) * kHeadDim;
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
                 uint32_t v[32];
                 ptx::tmem_ld32(acc_tm + q * 32, v);
                 ptx::tmem_wait_ld();
+                if (key < p.s_k) {
 #pragma unroll
-                for (int k = 0; k < 4; ++k) {
-                    const int cc = 4 * q + k;
-                    ptx::st_shared_v4(
-                        st_row + (cc >> 3) * kQTile64Bytes + (((cc & 7) ^ xr) << 4),
-                        ptx::pack_bf16x2(__uint_as_float(v[8 * k]) * f, __uint_as_float(v[8 * k + 1]) * f),
-                        ptx::pack_bf16x2(__uint_as_float(v[8 * k + 2]) * f, __uint_as_float(v[8 * k + 3]) * f),
-                        ptx::pack_bf16x2(__uint_as_float(v[8 * k + 4]) * f, __uint_as_float(v[8 * k + 5]) * f),
-                        ptx::pack_bf16x2(__uint_as_float(v[8 * k + 6]) * f, __uint_as_float(v[8 * k + 7]) * f));
+                    for (int k = 0; k < 4; ++k) {
+                        uint4 u;
+                        u.x = ptx::pack_bf16x2(__uint_as_float(v[8 * k]) * f, __uint_as_float(v[8 * k + 1]) * f);
+                        u.y = ptx::pack_bf16x2(__uint_as_float(v[8 * k + 2]) * f, __uint_as_float(v[8 * k + 3]) * f);
+                        u.z = ptx::pack_bf16x2(__uint_as_float(v[8 * k + 4]) * f, __uint_as_float(v[8 * k + 5]) * f);
+                        u.w = ptx::pack_bf16x2(__uint_as_float(v[8 * k + 6]) * f, __uint_as_float(v[8 * k + 7]) * f);
+                        *reinterpret_cast<uint4*>(row + q * 32 + 8 * k) = u;
+                    }
                 }
             }
             ptx::tc_fence_before();
-            ptx::fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) {
-                ptx::mbar_arrive(bar(L::bAccFree));
-                ptx::mbar_arrive(bar(L::bStaged + w));
-            }
-            if (r == 0) {
-                if (!wait_bar(bar(L::bStaged + w), items & 1, wc)) return;
-                const CUtensorMap* tm = w ? &tm_dk : &tm_dv;
-                ptx::tma_store_4d(tm, wg_base, 0, c.g, c.kb * kBlockN, c.b);
-                ptx::tma_store_4d(tm, wg_base + kQTile64Bytes, 64, c.g, c.kb * kBlockN, c.b);
-                ptx::bulk_commit_group();
-                ptx::bulk_wait_group_read0();
-                ptx::mbar_arrive(bar(L::bStored + w));
-            }
-            // This warpgroup's tiles are rewritten by its next step only
-            // after TMA has read the staged rows.
-            if (!wait_bar_warp(bar(L::bStored + w), items & 1, wc)) return;
+            if (lane == 0) ptx::mbar_arrive(bar(L::bAccFree));
             ++items;
         }
-        if (r == 0) ptx::bulk_wait_group0();
     }
 
     ptx::tc_fence_before();
