@@ -306,7 +306,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the issue loop; one elected lane issues.
+        {
             constexpr uint32_t kIdS = idesc_bf16_f32(kBlockM, kBlockN, 0, 0);    // Q K^T, dO V^T
             constexpr uint32_t kIdDq = idesc_bf16_f32(kBlockM, kHeadDim, 0, 1);  // dS K (K MN-major)
             const uint32_t q_lo = desc_lo_sw128(sbase + L::kQ, 16);
@@ -324,7 +325,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < kHeadDim / 16; ++k) {
                     const uint32_t off = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
-                    ptx::mma_ss(d_tm, desc_from_lo(a_lo + off), desc_from_lo(b_lo + off), kIdS,
+                    ptx::mma_ss_warp(d_tm, desc_from_lo(a_lo + off), desc_from_lo(b_lo + off), kIdS,
                                 k > 0 ? 1u : 0u);
                 }
             };
@@ -333,38 +334,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             // and dQ(j) runs while the compute warps start on block j + 1.
             auto scores = [&](uint32_t gs) -> bool {
                 const uint32_t ks = k_used % kStages;
-                if (!wait_bar(bar(L::bKFull + ks), (k_used / kStages) & 1, wc)) return false;
-                if (gs > 0 && !wait_bar(bar(L::bSFree), (gs - 1) & 1, wc)) return false;
+                if (!wait_bar_warp(bar(L::bKFull + ks), (k_used / kStages) & 1, wc)) return false;
+                if (gs > 0 && !wait_bar_warp(bar(L::bSFree), (gs - 1) & 1, wc)) return false;
                 ptx::tc_fence_after();
                 gemm_kmajor(s_tm, q_lo, k_lo + ((ks * kTileBytes) >> 4));
-                ptx::mma_commit(bar(L::bSFull));
+                ptx::mma_commit_warp(bar(L::bSFull));
                 ++k_used;  // K(j) stays in its slot until dQ(j) has read it
                 return true;
             };
             auto dprobs = [&](uint32_t gs) -> bool {
                 const uint32_t vs = v_used % kStages;
-                if (!wait_bar(bar(L::bVFull + vs), (v_used / kStages) & 1, wc)) return false;
-                if (gs > 0 && !wait_bar(bar(L::bPFree), (gs - 1) & 1, wc)) return false;
+                if (!wait_bar_warp(bar(L::bVFull + vs), (v_used / kStages) & 1, wc)) return false;
+                if (gs > 0 && !wait_bar_warp(bar(L::bPFree), (gs - 1) & 1, wc)) return false;
                 ptx::tc_fence_after();
                 gemm_kmajor(dp_tm, do_lo, v_lo + ((vs * kTileBytes) >> 4));
-                ptx::mma_commit(bar(L::bPFull));
-                ptx::mma_commit(bar(L::bVEmpty + vs));
+                ptx::mma_commit_warp(bar(L::bPFull));
+                ptx::mma_commit_warp(bar(L::bVEmpty + vs));
                 ++v_used;
                 return true;
             };
             uint32_t k_freed = 0;  // K tiles released after their dQ
             Cursor c;
             for (c.start(p); ok && c.valid(p); c.next(p)) {
-                if (!(ok = wait_bar(bar(L::bQFull), items & 1, wc))) break;
+                if (!(ok = wait_bar_warp(bar(L::bQFull), items & 1, wc))) break;
                 // dQ of the previous item must have been read out of TMEM.
-                if (items > 0 && !(ok = wait_bar(bar(L::bDqFree), (items - 1) & 1, wc))) break;
+                if (items > 0 && !(ok = wait_bar_warp(bar(L::bDqFree), (items - 1) & 1, wc))) break;
                 ++items;
                 if (!(ok = scores(steps) && dprobs(steps))) break;
                 for (int j = 0; j < c.n && ok; ++j) {
                     const uint32_t gs = steps + j;
                     if (j + 1 < c.n && !(ok = scores(gs + 1))) break;
                     // dQ += dS K once dS is in shared memory.
-                    if (!(ok = wait_bar(bar(L::bDsFull), gs & 1, wc))) break;
+                    if (!(ok = wait_bar_warp(bar(L::bDsFull), gs & 1, wc))) break;
                     ptx::tc_fence_after();
                     const uint32_t ks = k_freed % kStages;
                     const uint32_t kb = kmn_lo + ((ks * kTileBytes) >> 4);
@@ -373,21 +374,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                         // A = dS (K-major like Q); B = K, MN-major (head dim
                         // contiguous): 16 keys = 2 KiB per step.
                         const uint32_t off = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
-                        ptx::mma_ss(dq_tm, desc_from_lo(ds_lo + off),
+                        ptx::mma_ss_warp(dq_tm, desc_from_lo(ds_lo + off),
                                     desc_from_lo(kb + ((k * 2048) >> 4)), kIdDq,
                                     (j > 0 || k > 0) ? 1u : 0u);
                     }
-                    ptx::mma_commit(bar(L::bDsFree));
-                    ptx::mma_commit(bar(L::bKEmpty + ks));
+                    ptx::mma_commit_warp(bar(L::bDsFree));
+                    ptx::mma_commit_warp(bar(L::bKEmpty + ks));
                     ++k_freed;
                     if (j + 1 < c.n && !(ok = dprobs(gs + 1))) break;
                 }
                 if (!ok) break;
                 steps += c.n;
-                ptx::mma_commit(bar(L::bQEmpty));
-                ptx::mma_commit(bar(L::bDqFull));
+                ptx::mma_commit_warp(bar(L::bQEmpty));
+                ptx::mma_commit_warp(bar(L::bDqFull));
             }
-            ptx::mma_commit(bar(L::bDrain));
+            ptx::mma_commit_warp(bar(L::bDrain));
             wait_slow(bar(L::bDrain), 0, wc, false);
         }
         __syncwarp();
@@ -760,7 +761,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
     } else if (warp == kMmaWarp) {
         // ============================================================ MMA issuer
-        if (lane == 0) {
+        // The whole warp runs the issue loop; one elected lane issues.
+        {
             constexpr uint32_t kIdS = idesc_bf16_f32(kBlockN, kBlockM, 0, 0);     // K Q^T, V dO^T
             constexpr uint32_t kIdAcc = idesc_bf16_f32(kBlockN, kHeadDim, 0, 1);  // P^T dO, dS^T Q
             const uint32_t k_lo = desc_lo_sw128(sbase + L::kK, 16);
@@ -772,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < kHeadDim / 16; ++k) {
                     const uint32_t o = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
-                    ptx::mma_ss(d_tm, desc_from_lo(a_lo + o), desc_from_lo(b_lo + o), kIdS,
+                    ptx::mma_ss_warp(d_tm, desc_from_lo(a_lo + o), desc_from_lo(b_lo + o), kIdS,
                                 k > 0 ? 1u : 0u);
                 }
             };
@@ -785,7 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t b_lo = desc_lo_sw128(b_addr, kHalfTileBytes);
 #pragma unroll
                 for (int k = 0; k < kBlockM / 16; ++k)
-                    ptx::mma_ts(d_tm, a_tm + (k >> 2) * 64 + (k & 3) * 8,
+                    ptx::mma_ts_warp(d_tm, a_tm + (k >> 2) * 64 + (k & 3) * 8,
                                 desc_from_lo(b_lo + ((k * 2048) >> 4)), kIdAcc,
                                 (acc || k > 0) ? 1u : 0u);
             };
@@ -797,21 +799,21 @@ __global__ void __launch_bounds__(kThreads, 1)
             // new item's first S^T / dP^T also waits for its K / V; the last
             // S^T / dP^T of an item releases K / V for the next one.
             auto issue_s = [&](uint32_t u, bool first, bool last) -> bool {
-                if (first && !wait_bar(bar(L::bKFull), kv & 1, wc)) return false;
-                if (!wait_bar(bar(L::bQFull + u % kStages), (u / kStages) & 1, wc)) return false;
+                if (first && !wait_bar_warp(bar(L::bKFull), kv & 1, wc)) return false;
+                if (!wait_bar_warp(bar(L::bQFull + u % kStages), (u / kStages) & 1, wc)) return false;
                 ptx::tc_fence_after();
                 gemm_t(tmem + kTmS, k_lo, q_addr(u));
-                ptx::mma_commit(bar(L::bSFull));
-                if (last) ptx::mma_commit(bar(L::bKEmpty));
+                ptx::mma_commit_warp(bar(L::bSFull));
+                if (last) ptx::mma_commit_warp(bar(L::bKEmpty));
                 return true;
             };
             auto issue_dp = [&](uint32_t u, bool first, bool last) -> bool {
-                if (first && !wait_bar(bar(L::bVFull), kv & 1, wc)) return false;
-                if (!wait_bar(bar(L::bOFull + u % kStages), (u / kStages) & 1, wc)) return false;
+                if (first && !wait_bar_warp(bar(L::bVFull), kv & 1, wc)) return false;
+                if (!wait_bar_warp(bar(L::bOFull + u % kStages), (u / kStages) & 1, wc)) return false;
                 ptx::tc_fence_after();
                 gemm_t(tmem + kTmDP, v_lo, do_addr(u));
-                ptx::mma_commit(bar(L::bPFull));
-                if (last) ptx::mma_commit(bar(L::bVEmpty));
+                ptx::mma_commit_warp(bar(L::bPFull));
+                if (last) ptx::mma_commit_warp(bar(L::bVEmpty));
                 return true;
             };
             if (c.valid(p)) {
@@ -821,12 +823,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 while (ok) {
                     // Step gs (step s of n of the current item).  P^T(gs) in
                     // TMEM over S^T: dV += P^T dO.
-                    if (!(ok = wait_bar(bar(L::bPTFull), gs & 1, wc))) break;
-                    if (s == 0 && items > 0 && !(ok = wait_bar(bar(L::bAccFree), (items - 1) & 1, wc)))
+                    if (!(ok = wait_bar_warp(bar(L::bPTFull), gs & 1, wc))) break;
+                    if (s == 0 && items > 0 && !(ok = wait_bar_warp(bar(L::bAccFree), (items - 1) & 1, wc)))
                         break;
                     ptx::tc_fence_after();
                     gemm_acc(tmem + kTmDV, tmem + kTmS, do_addr(gs), s > 0);
-                    ptx::mma_commit(bar(L::bOEmpty + gs % kStages));
+                    ptx::mma_commit_warp(bar(L::bOEmpty + gs % kStages));
                     // The next step's S^T overwrites P^T(gs) only after the
                     // dV products above (the tensor core runs in issue order).
                     Cursor cn = c;
@@ -839,12 +841,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const bool more = cn.valid(p);
                     if (more && !(ok = issue_s(gs + 1, sn == 0, sn == nn - 1))) break;
                     // dS^T(gs) in TMEM over dP^T: dK += dS^T Q.
-                    if (!(ok = wait_bar(bar(L::bDSTFull), gs & 1, wc))) break;
+                    if (!(ok = wait_bar_warp(bar(L::bDSTFull), gs & 1, wc))) break;
                     ptx::tc_fence_after();
                     gemm_acc(tmem + kTmDK, tmem + kTmDP, q_addr(gs), s > 0);
-                    ptx::mma_commit(bar(L::bQEmpty + gs % kStages));
+                    ptx::mma_commit_warp(bar(L::bQEmpty + gs % kStages));
                     if (s == n - 1) {
-                        ptx::mma_commit(bar(L::bAccFull));
+                        ptx::mma_commit_warp(bar(L::bAccFull));
                         ++items;
                     }
                     if (more && !(ok = issue_dp(gs + 1, sn == 0, sn == nn - 1))) break;
@@ -856,7 +858,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     ++gs;
                 }
             }
-            ptx::mma_commit(bar(L::bDrain));
+            ptx::mma_commit_warp(bar(L::bDrain));
             wait_slow(bar(L::bDrain), 0, wc, false);
         }
         __syncwarp();
