@@ -541,14 +541,14 @@ extern "C" int attn_bwd(const void* q, const void* k, const void* v, const void*
     p.scale_log2 = static_cast<float>(static_cast<double>(scale) * 1.4426950408889634);
     float* Lw = static_cast<float*>(workspace);
     float* Dw = Lw + static_cast<size_t>(batch) * h_q * p.s_q_pad;
-    p.L = Lw;
+    p.NL = Lw;
     p.D = Dw;
     p.dk = static_cast<__nv_bfloat16*>(dk);
     p.dv = static_cast<__nv_bfloat16*>(dv);
     p.timeout_ns = g_timeout_ns;
     p.status = st->status;
 
-    // 1. D = rowsum(dO * O) and L = LSE log2(e), padded per head.
+    // 1. D = rowsum(dO * O) and -L = -LSE log2(e), padded per head.
     bwd::PrepParams a{static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout),
                       lse, Lw, Dw, batch, h_q, s_q, p.s_q_pad};
     const size_t rows = static_cast<size_t>(batch) * h_q * p.s_q_pad;

@@ -11,8 +11,8 @@
 //     dQ   = scale dS K,   dK = scale dS^T Q,   dV = P^T dO
 //
 // Three launches:
-//   attn_bwd_prep_kernel  -- D and L per query row (memory-bound), written
-//                            to a padded workspace (padding rows: L = +inf,
+//   attn_bwd_prep_kernel  -- D and -L per query row (memory-bound), written
+//                            to a padded workspace (padding rows: -L = -inf,
 //                            D = 0, so they carry weight 0);
 //   attn_bwd_dq_kernel    -- one CTA item per 128-row query block
 //                            (persistent): Q and dO stay in shared memory,
@@ -38,6 +38,8 @@
 // atomics: every output element is written once, by one CTA, and the result
 // is bit-for-bit reproducible.
 #pragma once
+
+#include <type_traits>
 
 #include "attn_common.cuh"
 
@@ -66,7 +68,7 @@ struct BwdParams {
     FastDiv div_h_kv;      // h_kv
     float scale;           // dQ, dK factor
     float scale_log2;      // scale * log2(e)
-    const float* L;        // [batch][h_q][s_q_pad]  LSE * log2(e) (+inf padding)
+    const float* NL;       // [batch][h_q][s_q_pad]  -LSE * log2(e) (-inf padding)
     const float* D;        // [batch][h_q][s_q_pad]  rowsum(dO * O) (0 padding)
     __nv_bfloat16* dk;     // [batch][s_k][h_kv][128] outputs of the dK/dV kernel
     __nv_bfloat16* dv;
@@ -76,13 +78,14 @@ struct BwdParams {
 
 // ------------------------------------------------------------------ prep
 // One warp per query row: D = sum_c dO[c] O[c] (BF16 in, FP32 sum) and
-// L = LSE * log2(e); the rows s_q .. s_q_pad - 1 of each head get L = +inf
-// and D = 0.
+// -L = -LSE * log2(e) (stored negated so the exponent 2^(S c - L) is one
+// fused multiply-add); the rows s_q .. s_q_pad - 1 of each head get
+// -L = -inf and D = 0.
 struct PrepParams {
     const __nv_bfloat16* o;
     const __nv_bfloat16* dout;
     const float* lse;
-    float* L;
+    float* NL;
     float* D;
     int batch, h_q, s_q, s_q_pad;
 };
@@ -99,7 +102,7 @@ __global__ void __launch_bounds__(kPrepThreads) attn_bwd_prep_kernel(const PrepP
         const int i = static_cast<int>(r - bh * a.s_q_pad);
         if (i >= a.s_q) {
             if (lane == 0) {
-                a.L[r] = CUDART_INF_F;
+                a.NL[r] = -CUDART_INF_F;
                 a.D[r] = 0.f;
             }
             continue;
@@ -123,7 +126,7 @@ __global__ void __launch_bounds__(kPrepThreads) attn_bwd_prep_kernel(const PrepP
         for (int sh = 16; sh > 0; sh >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, sh);
         if (lane == 0) {
             a.D[r] = acc;
-            a.L[r] = a.lse[bh * a.s_q + i] * 1.4426950408889634f;
+            a.NL[r] = a.lse[bh * a.s_q + i] * -1.4426950408889634f;
         }
     }
 }
@@ -408,13 +411,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             sbase + L::kDS + half * kHalfTileBytes + (r >> 3) * 1024 + (r & 7) * 128;
         const uint32_t xr = static_cast<uint32_t>(r & 7);
         const float c2 = p.scale_log2;
+        const uint64_t c2c2 = ptx::f2_pack(c2, c2);
         uint32_t items = 0, steps = 0;
         Cursor c;
         for (c.start(p); c.valid(p); c.next(p)) {
             const int row = c.qb * kBlockM + r;
             const size_t stat = (static_cast<size_t>(c.b) * p.h_q + c.h) * p.s_q_pad + row;
-            const float Lr = p.L[stat];  // +inf past s_q: P = 0
+            const float NLr = p.NL[stat];  // -inf past s_q: P = 0
             const float Dr = p.D[stat];
+            const uint64_t nl2 = ptx::f2_pack(NLr, NLr), nd2 = ptx::f2_pack(-Dr, -Dr);
             for (int j = 0; j < c.n; ++j, ++steps) {
                 const int kv0 = (c.kb_lo + j) * kBlockN + 64 * half;  // this half's first key
                 // Visible keys of this row inside the block: [lo, hi).
@@ -436,11 +441,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 ptx::tc_fence_before();
                 __syncwarp();
                 if (lane == 0) ptx::mbar_arrive(bar(L::bSFree));
+                // P = 2^(S c - L), pairs of columns in packed FP32; the mask
+                // is applied only where some row of the warp needs it (the
+                // diagonal and ragged blocks).
+                auto exps = [&](auto mask_tag) {
+                    constexpr bool kMask = decltype(mask_tag)::value;
 #pragma unroll
-                for (int k = 0; k < 64; ++k) {
-                    const float x = ptx::ex2(fmaf(pr[k], c2, -Lr));
-                    pr[k] = (k >= lo && k < hi) ? x : 0.f;
-                }
+                    for (int k = 0; k < 64; k += 2) {
+                        float x0, x1;
+                        ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(pr[k], pr[k + 1]), c2c2, nl2), x0, x1);
+                        x0 = ptx::ex2(x0);
+                        x1 = ptx::ex2(x1);
+                        if (kMask) {
+                            x0 = (k >= lo && k < hi) ? x0 : 0.f;
+                            x1 = (k + 1 >= lo && k + 1 < hi) ? x1 : 0.f;
+                        }
+                        pr[k] = x0;
+                        pr[k + 1] = x1;
+                    }
+                };
+                if (__any_sync(0xffffffffu, lo > 0 || hi < 64))
+                    exps(std::true_type{});
+                else
+                    exps(std::false_type{});
                 // dS = P (dP - D) -> BF16, into this warpgroup's half of the
                 // dS tile (K-major, 128-byte swizzle).
                 if (!wait_bar_warp(bar(L::bPFull), steps & 1, wc)) return;
@@ -454,8 +477,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                     uint32_t w[16];
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
-                        const float a = pr[q * 32 + 2 * k] * (__uint_as_float(dr[2 * k]) - Dr);
-                        const float b2 = pr[q * 32 + 2 * k + 1] * (__uint_as_float(dr[2 * k + 1]) - Dr);
+                        const uint64_t t = ptx::f2_add(
+                            ptx::f2_pack(__uint_as_float(dr[2 * k]), __uint_as_float(dr[2 * k + 1])), nd2);
+                        float a, b2;
+                        ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(pr[q * 32 + 2 * k], pr[q * 32 + 2 * k + 1]), t),
+                                       a, b2);
                         w[k] = ptx::pack_bf16x2(a, b2);
                     }
 #pragma unroll
@@ -704,7 +730,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const size_t stat =
                     (static_cast<size_t>(c.b) * p.h_q + h) * p.s_q_pad + qb * kBlockM;
                 const uint32_t ld = sbase + L::kLD + slot * L::kLDSlot;
-                ptx::bulk_load(ld, p.L + stat, kBlockM * 4, full);
+                ptx::bulk_load(ld, p.NL + stat, kBlockM * 4, full);
                 ptx::bulk_load(ld + kBlockM * 4, p.D + stat, kBlockM * 4, full);
                 return true;
             };
@@ -875,6 +901,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __nv_bfloat16* const out = w ? p.dk : p.dv;
         const float f = w ? p.scale : 1.f;
         const float c2 = p.scale_log2;
+        const uint64_t c2c2 = ptx::f2_pack(c2, c2), neg1 = ptx::f2_pack(-1.f, -1.f);
         uint32_t gs = 0, items = 0;
         Cursor c;
         for (c.start(p); c.valid(p); c.next(p)) {
@@ -893,7 +920,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const uint32_t sL = sbase + L::kLD + slot * L::kLDSlot + 4 * 64 * w;
                 const uint32_t sD = sL + kBlockM * 4;
                 float pt[64];
-                // L and D arrive with the step's Q tile; that slot is refilled
+                // -L and D arrive with the step's Q tile; that slot is refilled
                 // only after this step's dK products, which wait for dS^T.
                 if (!wait_bar_warp(bar(L::bQFull + slot), (gs / kStages) & 1, wc)) return;
                 if (!wait_bar_warp(bar(L::bSFull), gs & 1, wc)) return;
@@ -909,17 +936,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                         pt[32 + k] = __uint_as_float(s1[k]);
                     }
                 }
+                // P^T = 2^(S^T c - L), pairs of columns in packed FP32; the
+                // mask is applied only where some key row of the warp needs
+                // it (the diagonal steps of a causal or windowed launch).
+                auto exps = [&](auto mask_tag) {
+                    constexpr bool kMask = decltype(mask_tag)::value;
 #pragma unroll
-                for (int k4 = 0; k4 < 16; ++k4) {
-                    const float4 l4 = ptx::ld_shared_f4(sL + 16 * k4);  // same address: broadcast
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    for (int k4 = 0; k4 < 16; ++k4) {
+                        const float4 l4 = ptx::ld_shared_f4(sL + 16 * k4);  // -L, same address: broadcast
 #pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int k = 4 * k4 + e;
-                        const float x = ptx::ex2(fmaf(pt[k], c2, -lv[e]));
-                        pt[k] = (k >= lo && k <= hi) ? x : 0.f;
+                        for (int e = 0; e < 2; ++e) {
+                            const int k = 4 * k4 + 2 * e;
+                            float x0, x1;
+                            ptx::f2_unpack(ptx::f2_fma(ptx::f2_pack(pt[k], pt[k + 1]), c2c2,
+                                                       e ? ptx::f2_pack(l4.z, l4.w) : ptx::f2_pack(l4.x, l4.y)),
+                                           x0, x1);
+                            x0 = ptx::ex2(x0);
+                            x1 = ptx::ex2(x1);
+                            if (kMask) {
+                                x0 = (k >= lo && k <= hi) ? x0 : 0.f;
+                                x1 = (k + 1 >= lo && k + 1 <= hi) ? x1 : 0.f;
+                            }
+                            pt[k] = x0;
+                            pt[k + 1] = x1;
+                        }
                     }
-                }
+                };
+                if (__any_sync(0xffffffffu, lo > 0 || hi < 63))
+                    exps(std::true_type{});
+                else
+                    exps(std::false_type{});
                 // P^T in BF16 over the first 32 of this warpgroup's S^T
                 // columns (read above by this thread only).
                 {
@@ -944,11 +990,18 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                     for (int k4 = 0; k4 < 8; ++k4) {
                         const float4 d4 = ptx::ld_shared_f4(sD + 4 * (q * 32 + 4 * k4));
-                        const float dv4[4] = {d4.x, d4.y, d4.z, d4.w};
 #pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            const int k = 4 * k4 + e;
-                            pt[q * 32 + k] = pt[q * 32 + k] * (__uint_as_float(dr[k]) - dv4[e]);
+                        for (int e = 0; e < 2; ++e) {
+                            const int k = 4 * k4 + 2 * e;
+                            // (dP - D) by one packed FMA, then times P.
+                            const uint64_t t = ptx::f2_fma(
+                                e ? ptx::f2_pack(d4.z, d4.w) : ptx::f2_pack(d4.x, d4.y), neg1,
+                                ptx::f2_pack(__uint_as_float(dr[k]), __uint_as_float(dr[k + 1])));
+                            float a, b2;
+                            ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(pt[q * 32 + k], pt[q * 32 + k + 1]), t),
+                                           a, b2);
+                            pt[q * 32 + k] = a;
+                            pt[q * 32 + k + 1] = b2;
                         }
                     }
                 }
