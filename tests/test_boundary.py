@@ -43,6 +43,11 @@ def test_library_exports_every_declared_symbol(lib):
     assert set(declared_functions()) <= set(attn.EXPORTED)
 
 
+def test_every_bound_entry_point_is_declared():
+    missing = sorted(set(attn.EXPORTED) - set(declared_functions()))
+    assert not missing, f"bound but not declared in include/: {missing}"
+
+
 def test_strerror(lib):
     for code in range(6):
         assert attn.attn_strerror(code)
