@@ -156,14 +156,25 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
 
 /*
  * attn_fwd_host -- the same forward on HOST buffers: copies q, k, v to the
- * device (cudaMemcpyAsync on `stream`), runs attn_fwd, copies o and lse back,
- * and returns without synchronising (the caller synchronises `stream` before
- * reading o/lse; pinned host memory makes the copies asynchronous).
+ * device, runs the forward, copies o and lse back, and returns without
+ * synchronising (the caller synchronises `stream` before reading o/lse;
+ * pinned host memory makes the copies asynchronous).
  *
  *   q, k, v, o, lse   host pointers with the layouts of attn_fwd
  *   workspace         device buffer of at least
  *                     attn_fwd_host_workspace_bytes(...) bytes, 256-byte
  *                     aligned, owned by the caller
+ *
+ * Problems with at least two key/value heads and 32 MiB or more of inputs
+ * run in up to 8 groups of key/value heads (with their query heads, each
+ * group at least 16 MiB of inputs): a group's rows are copied in with strided
+ * copies on a host-to-device stream, its forward runs on `stream`, and its
+ * O and LSE go back on a device-to-host stream, so the copies of one group
+ * overlap the kernel of another.  The two copy streams and their events
+ * belong to the library (created on the first such call on each device).
+ * Ordering is that of `stream`: the call starts after the work already
+ * queued on it, and it waits for the call's last copy out, so synchronising
+ * `stream` covers everything.  Results are bit-identical to attn_fwd's.
  */
 int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
                   int batch, int h_q, int h_kv, int s_q, int s_k, int d,

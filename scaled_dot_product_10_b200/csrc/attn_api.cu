@@ -740,35 +740,151 @@ extern "C" size_t attn_fwd_host_workspace_bytes(int batch, int h_q, int h_kv, in
     return round_up(qb, 256) * 2 + round_up(kb, 256) * 2 + round_up(lb, 256);
 }
 
-extern "C" int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
-                             int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal,
-                             float scale, void* workspace, size_t workspace_bytes, void* stream) {
+// The host-buffer forward is pipelined: the problem is cut into up to
+// kHostChunks groups of key/value heads (each with its query heads), each
+// group a compact sub-problem in the workspace.  A group's inputs are copied
+// in with strided 2-D copies on an H2D stream, its forward runs on the
+// caller's stream once they have landed, and its O and LSE go back on a D2H
+// stream, so the copies of one group overlap the kernel of another.  Events
+// order the three streams; the caller's stream finally waits for the last
+// copy out, so synchronising it covers the whole call.
+constexpr int kHostChunks = 8;
+constexpr size_t kHostChunkMinBytes = size_t(16) << 20;  // smaller groups: fewer chunks
+
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t start = nullptr, done = nullptr;
+    cudaEvent_t in[kHostChunks] = {}, comp[kHostChunks] = {};
+    std::mutex mu;  // one call's enqueue sequence at a time per device
+};
+HostPipe g_pipe[kMaxDevices];
+
+int host_pipe(int dev, HostPipe** out) {
+    HostPipe& hp = g_pipe[dev];
+    if (!hp.ready) {
+        const unsigned fl = cudaEventDisableTiming;
+        if (cudaStreamCreateWithFlags(&hp.h2d, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaStreamCreateWithFlags(&hp.d2h, cudaStreamNonBlocking) != cudaSuccess ||
+            cudaEventCreateWithFlags(&hp.start, fl) != cudaSuccess ||
+            cudaEventCreateWithFlags(&hp.done, fl) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        for (int c = 0; c < kHostChunks; ++c)
+            if (cudaEventCreateWithFlags(&hp.in[c], fl) != cudaSuccess ||
+                cudaEventCreateWithFlags(&hp.comp[c], fl) != cudaSuccess)
+                return ATTN_ERR_CUDA;
+        hp.ready = true;
+    }
+    *out = &hp;
+    return ATTN_OK;
+}
+
+// Strided copy of `rows` rows of `width` bytes (a plain copy when the rows
+// are contiguous on both sides).
+cudaError_t copy_rows(void* dst, size_t dpitch, const void* src, size_t spitch, size_t width,
+                      size_t rows, cudaMemcpyKind kind, cudaStream_t s) {
+    if (dpitch == width && spitch == width)
+        return cudaMemcpyAsync(dst, src, width * rows, kind, s);
+    return cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, rows, kind, s);
+}
+
+// The host-buffer forward: pipelined on the library's streams, or (for the
+// allocation-free entry, which creates no streams or events) copy in, run
+// and copy out in order on the caller's stream alone.
+int host_forward(const void* q, const void* k, const void* v, void* o, float* lse, int batch,
+                 int h_q, int h_kv, int s_q, int s_k, int d, int causal, float scale,
+                 void* workspace, size_t workspace_bytes, void* stream, bool pipelined) {
     int rc = validate(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale);
     if (rc != ATTN_OK) return rc;
     if (!workspace) return ATTN_ERR_INVALID;
     if (!aligned(workspace, 256)) return ATTN_ERR_ALIGN;
     const size_t need = attn_fwd_host_workspace_bytes(batch, h_q, h_kv, s_q, s_k, d);
     if (workspace_bytes < need) return ATTN_ERR_INVALID;
-    const size_t qb = static_cast<size_t>(batch) * s_q * h_q * d * 2;
-    const size_t kb = static_cast<size_t>(batch) * s_k * h_kv * d * 2;
-    const size_t lb = static_cast<size_t>(batch) * h_q * s_q * 4;
-    char* w = static_cast<char*>(workspace);
-    char* dq = w;
-    char* dk = dq + round_up(qb, 256);
-    char* dv = dk + round_up(kb, 256);
-    char* d_o = dv + round_up(kb, 256);
-    float* dl = reinterpret_cast<float*>(d_o + round_up(qb, 256));
-    cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaMemcpyAsync(dq, q, qb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(dk, k, kb, cudaMemcpyHostToDevice, s) != cudaSuccess ||
-        cudaMemcpyAsync(dv, v, kb, cudaMemcpyHostToDevice, s) != cudaSuccess)
-        return ATTN_ERR_CUDA;
-    rc = attn_fwd(dq, dk, dv, d_o, dl, batch, h_q, h_kv, s_q, s_k, d, causal, scale, stream);
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ERR_CUDA;
+    DeviceState* st = nullptr;
+    rc = init_device(dev, &st);
     if (rc != ATTN_OK) return rc;
-    if (cudaMemcpyAsync(o, d_o, qb, cudaMemcpyDeviceToHost, s) != cudaSuccess ||
-        cudaMemcpyAsync(lse, dl, lb, cudaMemcpyDeviceToHost, s) != cudaSuccess)
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    HostPipe* hp = nullptr;
+    if (pipelined) {
+        std::lock_guard<std::mutex> lock(g_mutex);  // creation only: attn_fwd takes it too
+        rc = host_pipe(dev, &hp);
+        if (rc != ATTN_OK) return rc;
+    }
+    std::unique_lock<std::mutex> pipe_lock;
+    if (hp) pipe_lock = std::unique_lock<std::mutex>(hp->mu);
+    const cudaStream_t s_in = hp ? hp->h2d : s, s_out = hp ? hp->d2h : s;
+
+    const size_t row = static_cast<size_t>(d) * 2;  // bytes of one head's row
+    const size_t qb = static_cast<size_t>(batch) * s_q * h_q * row;
+    const size_t kb = static_cast<size_t>(batch) * s_k * h_kv * row;
+    int nc = !hp ? 1 : (h_kv < kHostChunks ? h_kv : kHostChunks);
+    while (nc > 1 && (qb + 2 * kb) / nc < kHostChunkMinBytes) --nc;
+    const int group = h_q / h_kv;
+    // Workspace: per group q | k | v | o (compact [b, s, heads, d]; every
+    // size a multiple of 256 bytes), then all groups' LSE [b, heads, s_q].
+    char* w = static_cast<char*>(workspace);
+    float* lse_all = reinterpret_cast<float*>(w + 2 * qb + 2 * kb);
+    if (hp && (cudaEventRecord(hp->start, s) != cudaSuccess ||
+               cudaStreamWaitEvent(hp->h2d, hp->start, 0) != cudaSuccess))
         return ATTN_ERR_CUDA;
+    size_t off = 0, loff = 0;
+    int g0 = 0;
+    for (int c = 0; c < nc; ++c) {
+        const int gc = h_kv / nc + (c < h_kv % nc ? 1 : 0);
+        const int hq0 = g0 * group, hqc = gc * group;
+        const size_t qc = static_cast<size_t>(batch) * s_q * hqc * row;
+        const size_t kc = static_cast<size_t>(batch) * s_k * gc * row;
+        char* dq = w + off;
+        char* dk = dq + qc;
+        char* dv = dk + kc;
+        char* d_o = dv + kc;
+        float* dl = lse_all + loff;
+        off += 2 * qc + 2 * kc;
+        loff += static_cast<size_t>(batch) * hqc * s_q;
+        const size_t q_rows = static_cast<size_t>(batch) * s_q;
+        const size_t k_rows = static_cast<size_t>(batch) * s_k;
+        const char* qh = static_cast<const char*>(q) + hq0 * row;
+        const char* kh = static_cast<const char*>(k) + g0 * row;
+        const char* vh = static_cast<const char*>(v) + g0 * row;
+        if (copy_rows(dq, hqc * row, qh, h_q * row, hqc * row, q_rows, cudaMemcpyHostToDevice,
+                      s_in) != cudaSuccess ||
+            copy_rows(dk, gc * row, kh, h_kv * row, gc * row, k_rows, cudaMemcpyHostToDevice,
+                      s_in) != cudaSuccess ||
+            copy_rows(dv, gc * row, vh, h_kv * row, gc * row, k_rows, cudaMemcpyHostToDevice,
+                      s_in) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        if (hp && (cudaEventRecord(hp->in[c], hp->h2d) != cudaSuccess ||
+                   cudaStreamWaitEvent(s, hp->in[c], 0) != cudaSuccess))
+            return ATTN_ERR_CUDA;
+        rc = attn_fwd(dq, dk, dv, d_o, dl, batch, hqc, gc, s_q, s_k, d, causal, scale, stream);
+        if (rc != ATTN_OK) return rc;
+        char* oh = static_cast<char*>(o) + hq0 * row;
+        char* lh = reinterpret_cast<char*>(lse) + static_cast<size_t>(hq0) * s_q * 4;
+        const size_t lw = static_cast<size_t>(hqc) * s_q * 4;
+        if (hp && (cudaEventRecord(hp->comp[c], s) != cudaSuccess ||
+                   cudaStreamWaitEvent(hp->d2h, hp->comp[c], 0) != cudaSuccess))
+            return ATTN_ERR_CUDA;
+        if (copy_rows(oh, h_q * row, d_o, hqc * row, hqc * row, q_rows, cudaMemcpyDeviceToHost,
+                      s_out) != cudaSuccess ||
+            copy_rows(lh, static_cast<size_t>(h_q) * s_q * 4, dl, lw, lw, batch,
+                      cudaMemcpyDeviceToHost, s_out) != cudaSuccess)
+            return ATTN_ERR_CUDA;
+        g0 += gc;
+    }
+    if (hp && (cudaEventRecord(hp->done, hp->d2h) != cudaSuccess ||
+               cudaStreamWaitEvent(s, hp->done, 0) != cudaSuccess))
+        return ATTN_ERR_CUDA;
+    g_last_launches = nc;
     return ATTN_OK;
+}
+
+extern "C" int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
+                             int batch, int h_q, int h_kv, int s_q, int s_k, int d, int causal,
+                             float scale, void* workspace, size_t workspace_bytes, void* stream) {
+    return host_forward(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale, workspace,
+                        workspace_bytes, stream, true);
 }
 
 extern "C" int attn_status(void* stream) {
@@ -853,6 +969,6 @@ extern "C" int attn_fwd_host_static(const void* q, const void* k, const void* v,
         }
         staging = g_static_staging_ptr[dev];
     }
-    return attn_fwd_host(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale, staging,
-                         ATTN_STATIC_STAGING_BYTES, stream);
+    return host_forward(q, k, v, o, lse, batch, h_q, h_kv, s_q, s_k, d, causal, scale, staging,
+                        ATTN_STATIC_STAGING_BYTES, stream, false);
 }

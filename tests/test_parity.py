@@ -198,6 +198,38 @@ def test_host_buffer_entry_point():
     assert_within(metrics(oo, ll, o_ref, l_ref), "host entry")
 
 
+@pytest.mark.parametrize("b,hq,hkv,s", [
+    (1, 16, 16, 8192),  # four groups of 4 key/value heads
+    (2, 12, 6, 4096),   # three groups of 2 (GQA)
+    (1, 10, 5, 8192),   # two uneven groups (3 and 2 key/value heads)
+])
+def test_host_buffer_pipelined_groups(b, hq, hkv, s):
+    """Large problems go through the host entry in groups of key/value heads
+    whose copies overlap the kernel of another group: every output must be
+    bit-identical to the device entry on the same inputs.  Two calls are
+    queued back to back on one workspace with different inputs, so the
+    second call's copies in must wait for the first call's kernels."""
+    q, k, v = make_qkv(b, hq, hkv, s, s, seed=6650 + hq)
+    q2 = make_qkv(b, hq, hkv, s, s, seed=6660 + hq)[0]
+    qh, q2h, kh, vh = q.pin_memory(), q2.pin_memory(), k.pin_memory(), v.pin_memory()
+    outs = [(torch.empty_like(qh).pin_memory(),
+             torch.empty((b, hq, s), dtype=torch.float32).pin_memory()) for _ in range(2)]
+    ws = torch.empty(attn.host_workspace_bytes(b, hq, hkv, s, s), dtype=torch.uint8, device="cuda")
+    attn.attn_fwd_host(qh, kh, vh, outs[0][0], outs[0][1], ws, causal=False, scale=SCALE)
+    attn.attn_fwd_host(q2h, kh, vh, outs[1][0], outs[1][1], ws, causal=True, scale=SCALE)
+    assert attn.attn_status() == attn.ATTN_OK
+    kd, vd = k.cuda(), v.cuda()
+    for (oh, lh), qq, causal in ((outs[0], q, False), (outs[1], q2, True)):
+        o_dev, l_dev = attn.attn_fwd(qq.cuda(), kd, vd, causal=causal, scale=SCALE)
+        assert attn.attn_status() == attn.ATTN_OK
+        assert torch.equal(oh, o_dev.cpu()), f"O differs (causal={causal})"
+        assert torch.equal(lh, l_dev.cpu()), f"LSE differs (causal={causal})"
+    rows = sample_rows(b, hq, s, 64, seed=6670 + hq)
+    o_ref, l_ref, _ = oracle.attn_fwd(q2, k, v, True, SCALE, rows=rows)
+    oo, ll = gather_rows(outs[1][0], outs[1][1], rows)
+    assert_within(metrics(oo, ll, o_ref, l_ref), "host entry, groups")
+
+
 def test_bounded_wait_reports_timeout_and_context_survives():
     assert attn.attn_status() == attn.ATTN_OK
     assert attn.selftest_wait_timeout(50_000_000) == attn.ATTN_OK  # 50 ms
