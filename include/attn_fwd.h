@@ -190,8 +190,10 @@ size_t attn_fwd_host_workspace_bytes(int batch, int h_q, int h_kv, int s_q, int 
  * and lse in a device array that the library itself declares at file scope
  * (ATTN_STATIC_STAGING_BYTES, held on every GPU that loads the library until
  * the process exits).  It calls no cudaMalloc/cudaFree or other allocating
- * routine.  The paper has no counterpart to this entry point: it is a
- * deployment convenience of this library.
+ * routine, and creates no streams or events: its copies in, forward and
+ * copies out run in order on `stream` alone (not grouped and overlapped as
+ * in attn_fwd_host).  The paper has no counterpart to this entry point: it
+ * is a deployment convenience of this library.
  *
  * Who needs it: code that may not allocate on the device at call time -- a
  * plugin handed only host arrays by an application that owns all device
