@@ -575,7 +575,7 @@ struct Smem {
     static constexpr int kV = kTileBytes;                    // V tile (A of dP^T = V dO^T)
     static constexpr int kQ = 2 * kTileBytes;                // ring of Q tiles (128 rows)
     static constexpr int kDO = kQ + kStages * kTileBytes;    // ring of dO tiles
-    static constexpr int kLD = kDO + kStages * kTileBytes;   // per Q slot: L[128], D[128]
+    static constexpr int kLD = kDO + kStages * kTileBytes;   // per Q slot: -L[128], D[128]
     static constexpr int kLDSlot = 2 * kBlockM * 4;
     static constexpr int kBars = kLD + kStages * kLDSlot;
     static constexpr int bKFull = 0, bKEmpty = 1, bVFull = 2, bVEmpty = 3, bQFull = 4,
