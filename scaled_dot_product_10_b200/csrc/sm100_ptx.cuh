@@ -206,18 +206,6 @@ __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
 
-// D(tmem) (+)= A(tmem) * B(smem desc)^T, kind::f16.  A is K-major in TMEM:
-// row m of the M = 128 tile in lane m, its 16 BF16 K-values packed in pairs
-// (even index in the low half) over 8 consecutive 32-bit columns.
-__device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                       uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate));
-}
-
 // Whole-warp forms of the issue instructions: every lane of a converged warp
 // executes them and one lane chosen by elect.sync issues.  Issuing from one
 // lane inside a divergent branch measured slower on B200 while other warps
@@ -232,6 +220,10 @@ __device__ __forceinline__ void mma_ss_warp(uint32_t d_tmem, uint64_t a_desc, ui
         "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate));
 }
+// mma_ts_warp: D(tmem) (+)= A(tmem) * B(smem desc)^T, kind::f16.  A is
+// K-major in TMEM: row m of the M = 128 tile in lane m, its 16 BF16 K-values
+// packed in pairs (even index in the low half) over 8 consecutive 32-bit
+// columns.
 __device__ __forceinline__ void mma_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
                                             uint32_t idesc, uint32_t accumulate) {
     asm volatile(
