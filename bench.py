@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--cpu-seconds", type=float, default=10.0,
                     help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--reference-seconds", type=float, default=150.0,
+                    help="--impl reference: total oracle time the run is sized for")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -267,8 +269,7 @@ def run_reference(args, world, rank):
     if rank != 0:
         return 0
     w = WORKLOADS[args.workload]
-    budget = 150.0
-    per_step = budget / max(1, args.steps + args.warmup)
+    per_step = args.reference_seconds / max(1, args.steps + args.warmup)
     import oracle
     q, k, v = workload_qkv(w)
     times, flops_total = [], 0.0
