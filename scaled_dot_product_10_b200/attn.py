@@ -468,7 +468,13 @@ def attn_status(stream=None) -> int:
 
 
 def set_wait_timeout_ns(ns: int) -> None:
-    load_library().attn_set_wait_timeout_ns(int(ns))
+    """Bound on every device-side wait of kernels launched afterwards (0: the
+    default, 2 s)."""
+    if int(ns) < 0:
+        raise ValueError("the timeout is a non-negative number of nanoseconds")
+    rc = load_library().attn_set_wait_timeout_ns(int(ns))
+    if rc != ATTN_OK:
+        raise AttnError(rc, "attn_set_wait_timeout_ns")
 
 
 def selftest_wait_timeout(timeout_ns: int, stream=None) -> int:

@@ -286,3 +286,13 @@ def test_fp8_entry_validation(lib):
     assert f(A + 8, *ok[1:], 1.0, 1.0, 1.0, None) == attn.ATTN_ERR_ALIGN
     if not torch.cuda.is_available():
         assert f(*ok, 1.0, 1.0, 1.0, None) == attn.ATTN_ERR_CUDA
+
+
+def test_wait_timeout_setter(lib):
+    """Host-only: any bound is accepted and 0 restores the default."""
+    assert lib.attn_set_wait_timeout_ns(5_000_000_000) == attn.ATTN_OK
+    assert lib.attn_set_wait_timeout_ns(0) == attn.ATTN_OK
+    attn.set_wait_timeout_ns(3_000_000_000)
+    attn.set_wait_timeout_ns(0)
+    with pytest.raises(ValueError):
+        attn.set_wait_timeout_ns(-1)
