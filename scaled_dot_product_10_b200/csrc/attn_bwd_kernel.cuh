@@ -19,8 +19,9 @@
 //                            K/V tiles stream through a two-slot ring; per
 //                            key block S and dP on the tensor core (TMEM),
 //                            dS by two warpgroups (each 64 of the block's
-//                            keys, thread = row), dQ += dS K on the tensor
-//                            core;
+//                            keys, thread = row), written to TMEM in BF16;
+//                            dQ += dS K on the tensor core reads it there as
+//                            the A operand;
 //   attn_bwd_dkdv_kernel  -- one CTA item per 128-key block of a key/value
 //                            head: K and V stay in shared memory, 128-row
 //                            Q / dO tiles of every query head of the group
@@ -145,7 +146,7 @@ constexpr int kMmaWarp = 9;
 struct Smem {
     static constexpr int kQ = 0;                       // Q tile  (A of S = Q K^T)
     static constexpr int kDO = kTileBytes;             // dO tile (A of dP = dO V^T)
-    static constexpr int kDS = 2 * kTileBytes;         // dS (A of dQ += dS K); O staging
+    static constexpr int kOut = 2 * kTileBytes;        // dQ staging for the TMA store
     static constexpr int kK = 3 * kTileBytes;          // K ring (2)
     static constexpr int kV = 5 * kTileBytes;          // V ring (2)
     static constexpr int kBars = 7 * kTileBytes;
@@ -315,11 +316,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             constexpr uint32_t kIdDq = idesc_bf16_f32(kBlockM, kHeadDim, 0, 1);  // dS K (K MN-major)
             const uint32_t q_lo = desc_lo_sw128(sbase + L::kQ, 16);
             const uint32_t do_lo = desc_lo_sw128(sbase + L::kDO, 16);
-            const uint32_t ds_lo = desc_lo_sw128(sbase + L::kDS, 16);
             const uint32_t k_lo = desc_lo_sw128(sbase + L::kK, 16);
             const uint32_t kmn_lo = desc_lo_sw128(sbase + L::kK, kHalfTileBytes);
             const uint32_t v_lo = desc_lo_sw128(sbase + L::kV, 16);
-            const uint32_t s_tm = tmem, dp_tm = tmem + 128, dq_tm = tmem + 256;
+            // TMEM: S | dP | dQ | dS (BF16, the A operand of dQ += dS K) at
+            // columns 0, 128, 256, 384.
+            const uint32_t s_tm = tmem, dp_tm = tmem + 128, dq_tm = tmem + 256, ds_tm = tmem + 384;
             uint32_t k_used = 0, v_used = 0, items = 0, steps = 0;
             bool ok = true;
             // K-major operands: 8 K-steps of 16 BF16 (32 bytes) inside a
@@ -367,19 +369,20 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < c.n && ok; ++j) {
                     const uint32_t gs = steps + j;
                     if (j + 1 < c.n && !(ok = scores(gs + 1))) break;
-                    // dQ += dS K once dS is in shared memory.
+                    // dQ += dS K once dS is in TMEM.
                     if (!(ok = wait_bar_warp(bar(L::bDsFull), gs & 1, wc))) break;
                     ptx::tc_fence_after();
                     const uint32_t ks = k_freed % kStages;
                     const uint32_t kb = kmn_lo + ((ks * kTileBytes) >> 4);
 #pragma unroll
                     for (int k = 0; k < kBlockN / 16; ++k) {
-                        // A = dS (K-major like Q); B = K, MN-major (head dim
-                        // contiguous): 16 keys = 2 KiB per step.
-                        const uint32_t off = ((k >> 2) * kHalfTileBytes + (k & 3) * 32) >> 4;
-                        ptx::mma_ss_warp(dq_tm, desc_from_lo(ds_lo + off),
-                                    desc_from_lo(kb + ((k * 2048) >> 4)), kIdDq,
-                                    (j > 0 || k > 0) ? 1u : 0u);
+                        // A = dS from TMEM: 16 keys = 8 packed columns per
+                        // step (keys 0-63 written by warpgroup 0, 64-127 by
+                        // warpgroup 1); B = K, MN-major (head dim contiguous):
+                        // 16 keys = 2 KiB per step.
+                        ptx::mma_ts_warp(dq_tm, ds_tm + 8 * k,
+                                         desc_from_lo(kb + ((k * 2048) >> 4)), kIdDq,
+                                         (j > 0 || k > 0) ? 1u : 0u);
                     }
                     ptx::mma_commit_warp(bar(L::bDsFree));
                     ptx::mma_commit_warp(bar(L::bKEmpty + ks));
@@ -404,11 +407,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const uint32_t s_tm = tmem + lane_base + 64 * half,
                        dp_tm = tmem + lane_base + 128 + 64 * half,
-                       dq_tm = tmem + lane_base + 256 + 64 * half;
-        // This row's half of the dS tile: the tile's 64-column half `half`
-        // (16 KiB), chunk k of the half at ((k ^ (r % 8)) * 16).
-        const uint32_t ds_row =
-            sbase + L::kDS + half * kHalfTileBytes + (r >> 3) * 1024 + (r & 7) * 128;
+                       dq_tm = tmem + lane_base + 256 + 64 * half,
+                       ds_tm = tmem + lane_base + 384 + 32 * half;
+        // This row's half of the dQ staging tile: the tile's 64-column half
+        // `half` (16 KiB), chunk k of the half at ((k ^ (r % 8)) * 16).
+        const uint32_t out_row =
+            sbase + L::kOut + half * kHalfTileBytes + (r >> 3) * 1024 + (r & 7) * 128;
         const uint32_t xr = static_cast<uint32_t>(r & 7);
         const float c2 = p.scale_log2;
         const uint64_t c2c2 = ptx::f2_pack(c2, c2);
@@ -464,17 +468,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                     exps(std::true_type{});
                 else
                     exps(std::false_type{});
-                // dS = P (dP - D) -> BF16, into this warpgroup's half of the
-                // dS tile (K-major, 128-byte swizzle).
+                // dS = P (dP - D) -> BF16 pairs, into this warpgroup's 32
+                // TMEM columns of dS (its 64 keys, the A operand of dQ).
                 if (!wait_bar_warp(bar(L::bPFull), steps & 1, wc)) return;
                 if (steps > 0 && !wait_bar_warp(bar(L::bDsFree), (steps - 1) & 1, wc)) return;
                 ptx::tc_fence_after();
+                uint32_t ds[32];
 #pragma unroll
                 for (int q = 0; q < 2; ++q) {
                     uint32_t dr[32];
                     ptx::tmem_ld32(dp_tm + q * 32, dr);
                     ptx::tmem_wait_ld();
-                    uint32_t w[16];
 #pragma unroll
                     for (int k = 0; k < 16; ++k) {
                         const uint64_t t = ptx::f2_add(
@@ -482,17 +486,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                         float a, b2;
                         ptx::f2_unpack(ptx::f2_mul(ptx::f2_pack(pr[q * 32 + 2 * k], pr[q * 32 + 2 * k + 1]), t),
                                        a, b2);
-                        w[k] = ptx::pack_bf16x2(a, b2);
-                    }
-#pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int cc = 4 * q + k;  // chunk within this half
-                        ptx::st_shared_v4(ds_row + ((cc ^ xr) << 4), w[4 * k], w[4 * k + 1],
-                                          w[4 * k + 2], w[4 * k + 3]);
+                        ds[q * 16 + k] = ptx::pack_bf16x2(a, b2);
                     }
                 }
+                ptx::tmem_st32(ds_tm, ds);
+                ptx::tmem_wait_st();
                 ptx::tc_fence_before();
-                ptx::fence_proxy_async_smem();
                 __syncwarp();
                 if (lane == 0) {
                     ptx::mbar_arrive(bar(L::bPFree));
@@ -500,8 +499,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             // Epilogue: dQ * scale -> BF16 rows, each warpgroup its 64
-            // columns, staged in its half of the dS tile (free once the last
-            // dQ MMA has completed) and stored with TMA.
+            // columns, staged in its half of the staging tile and stored
+            // with TMA.
             if (!wait_bar_warp(bar(L::bDqFull), items & 1, wc)) return;
             ptx::tc_fence_after();
 #pragma unroll
@@ -517,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
                 for (int k = 0; k < 4; ++k) {
                     const int cc = 4 * q + k;
-                    ptx::st_shared_v4(ds_row + ((cc ^ xr) << 4), w[4 * k], w[4 * k + 1],
+                    ptx::st_shared_v4(out_row + ((cc ^ xr) << 4), w[4 * k], w[4 * k + 1],
                                       w[4 * k + 2], w[4 * k + 3]);
                 }
             }
@@ -530,15 +529,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (warp == 0 && lane == 0) {
                 if (!wait_bar(bar(L::bStaged), items & 1, wc)) return;
-                ptx::tma_store_4d(&tm_dq, sbase + L::kDS, 0, c.h, c.qb * kBlockM, c.b);
-                ptx::tma_store_4d(&tm_dq, sbase + L::kDS + kHalfTileBytes, 64, c.h,
+                ptx::tma_store_4d(&tm_dq, sbase + L::kOut, 0, c.h, c.qb * kBlockM, c.b);
+                ptx::tma_store_4d(&tm_dq, sbase + L::kOut + kHalfTileBytes, 64, c.h,
                                   c.qb * kBlockM, c.b);
                 ptx::bulk_commit_group();
                 ptx::bulk_wait_group_read0();
                 ptx::mbar_arrive(bar(L::bStored));
             }
-            // The dS tile is rewritten by the next item only after TMA has
-            // read the staged rows.
+            // The staging tile is rewritten by the next item only after TMA
+            // has read the staged rows.
             if (!wait_bar_warp(bar(L::bStored), items & 1, wc)) return;
             ++items;
         }
