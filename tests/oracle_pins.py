@@ -19,6 +19,7 @@ import math
 import os
 
 import numpy as np
+import scipy.special
 import torch
 
 import oracle
@@ -262,7 +263,9 @@ def pin_gqa_equals_repeated_mha(lib):
 def pin_torch_sdpa_f64(lib):
     """Independent library routine: torch's float64 CPU scaled_dot_product_attention
     (with is_causal and enable_gqa) gives the same O; the LSE matches
-    torch.logsumexp of the library matmul's scaled scores."""
+    scipy's logsumexp of the library matmul's scaled scores.  (torch's own
+    CPU logsumexp is not used: on bit-identical float64 scores it returned a
+    result 4.6e-10 off in about one process in twenty.)"""
     cases = [(2, 4, 4, 67, 16), (1, 4, 2, 45, 128), (2, 8, 1, 40, 32)]
     for b, h_q, h_kv, s, d in cases:
         q, k, v = make_qkv(b, h_q, h_kv, s, s, seed=100 + s, d=d)
@@ -279,8 +282,8 @@ def pin_torch_sdpa_f64(lib):
             sc = torch.matmul(qt, kr.transpose(-1, -2)) * scale
             if causal:
                 sc = sc.masked_fill(torch.ones(s, s, dtype=torch.bool).triu(1), float("-inf"))
-            want_lse = torch.logsumexp(sc, dim=-1).numpy()
-            assert np.max(np.abs(lse - want_lse)) < 1e-10, "LSE disagrees with torch.logsumexp"
+            want_lse = scipy.special.logsumexp(sc.numpy(), axis=-1)
+            assert np.max(np.abs(lse - want_lse)) < 1e-10, "LSE disagrees with scipy's logsumexp"
 
 
 def _closed_form(expr: str) -> float:
@@ -329,9 +332,9 @@ def _varlen_case(seed, lens_q, lens_k, h_q=4, h_kv=2, d=16):
 def pin_varlen_matches_block_diagonal_sdpa(lib):
     """A packed batch equals ONE attention over all packed tokens whose mask
     forbids every (query, key) pair of different sequences (and, causal,
-    keys past the row's own diagonal in its sequence): torch's float64 SDPA
-    with that explicit boolean mask, and torch.logsumexp of the masked
-    scores."""
+    keys past the row's own diagonal in its sequence; with a window of W,
+    also keys more than W before that diagonal): torch's float64 SDPA with
+    that explicit boolean mask, and scipy's logsumexp of the masked scores."""
     lens_q, lens_k = [5, 1, 9, 3], [7, 4, 9, 3]
     q, k, v, cu_q, cu_k = _varlen_case(31, lens_q, lens_k)
     h_q, h_kv = q.shape[1], k.shape[1]
@@ -340,10 +343,12 @@ def pin_varlen_matches_block_diagonal_sdpa(lib):
     pos_q = np.arange(cu_q[-1]) - cu_q[seq_q]
     pos_k = np.arange(cu_k[-1]) - cu_k[seq_k]
     off = (np.asarray(lens_k) - np.asarray(lens_q))[seq_q]
-    for causal in (False, True):
+    for causal, window in ((False, -1), (True, -1), (True, 0), (True, 3)):
         allow = seq_q[:, None] == seq_k[None, :]
         if causal:
             allow &= pos_k[None, :] <= (pos_q + off)[:, None]
+        if window >= 0:
+            allow &= pos_k[None, :] >= (pos_q + off - window)[:, None]
         mask = torch.from_numpy(allow)
         qt = q.double().permute(1, 0, 2)[None]                    # [1, h_q, Tq, d]
         kt = k.double().permute(1, 0, 2).repeat_interleave(h_q // h_kv, 0)[None]
@@ -351,10 +356,12 @@ def pin_varlen_matches_block_diagonal_sdpa(lib):
         want = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=mask,
                                                                 scale=0.3)
         scores = (qt @ kt.transpose(-1, -2)) * 0.3
-        want_lse = torch.logsumexp(scores.masked_fill(~mask, float("-inf")), dim=-1)
-        o, lse = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, causal, 0.3, lib=lib)
-        assert np.max(np.abs(o - want[0].permute(1, 0, 2).numpy())) < 1e-10, "varlen O"
-        assert np.max(np.abs(lse - want_lse[0].numpy())) < 1e-10, "varlen LSE"
+        want_lse = scipy.special.logsumexp(scores.masked_fill(~mask, float("-inf")).numpy(), axis=-1)
+        o, lse = oracle.attn_fwd_varlen(q, k, v, cu_q, cu_k, causal, 0.3, window_left=window,
+                                        lib=lib)
+        what = f"varlen causal={causal} window={window}"
+        assert np.max(np.abs(o - want[0].permute(1, 0, 2).numpy())) < 1e-10, what + ": O"
+        assert np.max(np.abs(lse - want_lse[0])) < 1e-10, what + ": LSE"
 
 
 def pin_varlen_sequences_are_independent(lib):

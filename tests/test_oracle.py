@@ -149,3 +149,48 @@ def test_planted_mistake_is_caught(tmp_path, name):
                    check=True)
     bad = failing_pins(oracle.load(str(so)))
     assert bad, f"planted mistake '{name}' passed every pin"
+
+
+# Planted mistakes in the oracle's packed-batch wrapper (Python): the
+# function's source is rewritten, compiled in the oracle module's namespace
+# and swapped in for the pins; each mutant must fail at least one pin.
+VARLEN_MUTANTS = {
+    "varlen_keys_at_query_offsets": ("kb[None, k0:k1], vb[None, k0:k1]",
+                                     "kb[None, q0:q1], vb[None, q0:q1]"),
+    "varlen_skips_last_sequence": ("for b in range(len(cu_q) - 1):",
+                                   "for b in range(len(cu_q) - 2):"),
+    "varlen_drops_window": ("window_left=window_left)", "window_left=-1)"),
+    "varlen_lse_rows_reversed": ("lse[:, q0:q1] = lb[0]", "lse[:, q0:q1] = lb[0][:, ::-1]"),
+    "varlen_heads_not_transposed": ("o[q0:q1] = ob[0].transpose(1, 0, 2)",
+                                    "o[q0:q1] = ob[0].reshape(o[q0:q1].shape)"),
+    "varlen_v_from_k": ("vb[None, k0:k1], causal", "kb[None, k0:k1], causal"),
+}
+
+
+def _rebuilt_varlen(old: str | None = None, new: str | None = None):
+    """oracle.attn_fwd_varlen recompiled from its source, with `old`
+    replaced by `new` (once) when given."""
+    import inspect
+    import textwrap
+
+    src = textwrap.dedent(inspect.getsource(oracle.attn_fwd_varlen))
+    if old is not None:
+        assert src.count(old) == 1, f"mutation site {old!r} not found"
+        src = src.replace(old, new)
+    ns = dict(vars(oracle))
+    exec(compile(src, "<varlen rebuilt>", "exec"), ns)  # noqa: S102
+    return ns["attn_fwd_varlen"]
+
+
+def test_rebuilt_varlen_passes_every_pin(lib, monkeypatch):
+    """Control for the mutants below: the unmodified source, rebuilt the
+    same way, fails no pin (so a mutant's failure is its mistake's)."""
+    monkeypatch.setattr(oracle, "attn_fwd_varlen", _rebuilt_varlen())
+    assert failing_pins(lib) == []
+
+
+@pytest.mark.parametrize("name", sorted(VARLEN_MUTANTS))
+def test_planted_varlen_mistake_is_caught(lib, monkeypatch, name):
+    monkeypatch.setattr(oracle, "attn_fwd_varlen", _rebuilt_varlen(*VARLEN_MUTANTS[name]))
+    bad = failing_pins(lib)
+    assert bad, f"planted mistake '{name}' passed every pin"
