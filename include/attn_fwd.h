@@ -25,6 +25,12 @@
  *
  * Every function returns an attn_status_t code.  On any error nothing is
  * written to o or lse.
+ *
+ * Device: every call launches on the calling thread's current CUDA device
+ * (cudaGetDevice).  Device buffers must be allocations on that device and
+ * `stream` one of its streams; the library does not look up where a pointer
+ * lives, so a buffer of another device is not detected.  The Python binding
+ * checks that the tensors of a call share one device and makes it current.
  */
 #ifndef SDPA10_ATTN_FWD_H
 #define SDPA10_ATTN_FWD_H

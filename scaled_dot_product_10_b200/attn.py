@@ -110,6 +110,32 @@ def _stream_obj(stream, device):
     return stream
 
 
+def _cuda_device(stream, **tensors):
+    """The one CUDA device every tensor of a call is on.  The library
+    launches on the calling thread's current device, so each call runs under
+    this device (see :func:`_on_device`); a torch stream given for the call
+    must belong to it."""
+    dev = None
+    for name, t in tensors.items():
+        if not t.is_cuda:
+            raise ValueError(f"{name} must be a CUDA tensor")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError(f"{name} is on {t.device}, the call's other tensors on {dev}")
+    sdev = getattr(stream, "device", None)
+    if dev is not None and sdev is not None and sdev != dev:
+        raise ValueError(f"stream belongs to {sdev}, the tensors to {dev}")
+    return dev
+
+
+def _on_device(dev):
+    """Context making ``dev`` the current device for the library call (and
+    for the default stream, torch's current stream on that device)."""
+    import torch
+    return torch.cuda.device(dev)
+
+
 def _alloc_on(stream, device, fn):
     """Allocate with ``fn()`` on the launch stream, so the caching allocator
     never hands a buffer that a kernel of this call still uses to work queued
@@ -148,20 +174,39 @@ def _check_qkv(q, k, v):
     return b, s_q, h_q, h_kv, s_k, d
 
 
+def _out(ref, t, name, shape, dtype, stream):
+    """Check a caller-supplied output, or allocate it on the launch stream."""
+    if t is None:
+        import torch
+        return _alloc_on(stream, ref.device,
+                         lambda: torch.empty(shape, dtype=dtype, device=ref.device))
+    _check_out(t, name, shape, dtype, ref.device)
+    return t
+
+
 def _outputs(q, o, lse, o_shape, lse_shape, stream, o_dtype=None):
     """Check caller-supplied outputs, or allocate them on the launch stream."""
     import torch
-    o_dtype = o_dtype or torch.bfloat16
-    if o is None:
-        o = _alloc_on(stream, q.device, lambda: torch.empty(o_shape, dtype=o_dtype, device=q.device))
-    else:
-        _check_out(o, "o", o_shape, o_dtype, q.device)
-    if lse is None:
-        lse = _alloc_on(stream, q.device,
-                        lambda: torch.empty(lse_shape, dtype=torch.float32, device=q.device))
-    else:
-        _check_out(lse, "lse", lse_shape, torch.float32, q.device)
-    return o, lse
+    return (_out(q, o, "o", o_shape, o_dtype or torch.bfloat16, stream),
+            _out(q, lse, "lse", lse_shape, torch.float32, stream))
+
+
+def _workspace(ref, workspace, nbytes, stream):
+    """A caller's workspace (contiguous, on the inputs' device, at least
+    ``nbytes``; the C side checks the size too) or one allocated on the
+    launch stream, whose memory is then not reused before the call's kernels
+    finish even though it is dropped on return."""
+    if workspace is None:
+        import torch
+        return _alloc_on(stream, ref.device,
+                         lambda: torch.empty(nbytes, dtype=torch.uint8, device=ref.device))
+    if workspace.device != ref.device or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on the inputs' device")
+    return workspace
+
+
+def _nbytes(t) -> int:
+    return t.numel() * t.element_size()
 
 
 def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, lse=None,
@@ -169,19 +214,17 @@ def attn_fwd(q, k, v, causal: bool = False, scale: float | None = None, o=None, 
     """O, LSE = attention forward on CUDA tensors [batch, seq, heads, 128] (BF16).
 
     Returns (o [b, s_q, h_q, 128] BF16, lse [b, h_q, s_q] FP32).  Asynchronous
-    on ``stream`` (default: torch's current stream).
+    on ``stream`` (default: torch's current stream on the tensors' device).
     """
-    import torch
     b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        if not t.is_cuda:
-            raise ValueError(f"{name} must be a CUDA tensor")
+    dev = _cuda_device(stream, q=q, k=k, v=v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
-    rc = load_library().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                 lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d, int(bool(causal)),
-                                 float(scale), _stream_handle(stream))
+    with _on_device(dev):
+        o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
+        rc = load_library().attn_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                     lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
+                                     int(bool(causal)), float(scale), _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd")
     return o, lse
@@ -193,15 +236,15 @@ def attn_fwd_window(q, k, v, window_left: int, scale: float | None = None, o=Non
     i + s_k - s_q - window_left .. i + s_k - s_q.  Returns (o, lse) as
     :func:`attn_fwd`."""
     b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        if not t.is_cuda:
-            raise ValueError(f"{name} must be a CUDA tensor")
+    dev = _cuda_device(stream, q=q, k=k, v=v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
-    rc = load_library().attn_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                        lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
-                                        int(window_left), float(scale), _stream_handle(stream))
+    with _on_device(dev):
+        o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
+        rc = load_library().attn_fwd_window(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            o.data_ptr(), lse.data_ptr(), b, h_q, h_kv, s_q,
+                                            s_k, d, int(window_left), float(scale),
+                                            _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_window")
     return o, lse
@@ -221,6 +264,8 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
     for name, t in (("cu_seqlens_q", cu_seqlens_q), ("cu_seqlens_k", cu_seqlens_k)):
         if t.dtype != torch.int32 or t.dim() != 1 or not t.is_contiguous() or not t.is_cuda:
             raise ValueError(f"{name} must be a contiguous CUDA int32 vector")
+    dev = _cuda_device(stream, q=q, k=k, v=v, cu_seqlens_q=cu_seqlens_q,
+                       cu_seqlens_k=cu_seqlens_k)
     total_q, h_q, d = q.shape
     total_k, h_kv, dk = k.shape
     if tuple(v.shape) != tuple(k.shape) or dk != d:
@@ -230,13 +275,15 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q: int, max_
         raise ValueError("cu_seqlens_q and cu_seqlens_k need batch + 1 entries")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    o, lse = _outputs(q, o, lse, (total_q, h_q, d), (h_q, total_q), stream)
-    rc = load_library().attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                        lse.data_ptr(), cu_seqlens_q.data_ptr(),
-                                        cu_seqlens_k.data_ptr(), batch, int(max_seqlen_q),
-                                        int(max_seqlen_k), total_q, total_k, h_q, h_kv, d,
-                                        int(bool(causal)), int(window_left), float(scale),
-                                        _stream_handle(stream))
+    with _on_device(dev):
+        o, lse = _outputs(q, o, lse, (total_q, h_q, d), (h_q, total_q), stream)
+        rc = load_library().attn_fwd_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                            o.data_ptr(), lse.data_ptr(),
+                                            cu_seqlens_q.data_ptr(), cu_seqlens_k.data_ptr(),
+                                            batch, int(max_seqlen_q), int(max_seqlen_k),
+                                            total_q, total_k, h_q, h_kv, d, int(bool(causal)),
+                                            int(window_left), float(scale),
+                                            _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_varlen")
     return o, lse
@@ -253,27 +300,23 @@ def attn_bwd(q, k, v, o, lse, dout, causal: bool = False, scale: float | None = 
     incoming gradient dout (shaped like o).  Three launches on ``stream``."""
     import torch
     b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        if not t.is_cuda:
-            raise ValueError(f"{name} must be a CUDA tensor")
-    _check_out(o, "o", (b, s_q, h_q, d), torch.bfloat16, q.device)
-    _check_out(dout, "dout", (b, s_q, h_q, d), torch.bfloat16, q.device)
-    _check_out(lse, "lse", (b, h_q, s_q), torch.float32, q.device)
+    dev = _cuda_device(stream, q=q, k=k, v=v)
+    _check_out(o, "o", (b, s_q, h_q, d), torch.bfloat16, dev)
+    _check_out(dout, "dout", (b, s_q, h_q, d), torch.bfloat16, dev)
+    _check_out(lse, "lse", (b, h_q, s_q), torch.float32, dev)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    dq, _ = _outputs(q, dq, None, (b, s_q, h_q, d), (1,), stream)
-    dk, _ = _outputs(k, dk, None, (b, s_k, h_kv, d), (1,), stream)
-    dv, _ = _outputs(v, dv, None, (b, s_k, h_kv, d), (1,), stream)
-    if workspace is None:
-        nbytes = bwd_workspace_bytes(b, h_q, s_q)
-        workspace = _alloc_on(stream, q.device,
-                              lambda: torch.empty(nbytes, dtype=torch.uint8, device=q.device))
-    rc = load_library().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                 dout.data_ptr(), lse.data_ptr(), dq.data_ptr(), dk.data_ptr(),
-                                 dv.data_ptr(), b, h_q, h_kv, s_q, s_k, d, int(bool(causal)),
-                                 int(window_left), float(scale), workspace.data_ptr(),
-                                 workspace.numel() * workspace.element_size(),
-                                 _stream_handle(stream))
+    with _on_device(dev):
+        dq = _out(q, dq, "dq", (b, s_q, h_q, d), torch.bfloat16, stream)
+        dk = _out(q, dk, "dk", (b, s_k, h_kv, d), torch.bfloat16, stream)
+        dv = _out(q, dv, "dv", (b, s_k, h_kv, d), torch.bfloat16, stream)
+        workspace = _workspace(q, workspace, bwd_workspace_bytes(b, h_q, s_q), stream)
+        rc = load_library().attn_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                     dout.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+                                     dk.data_ptr(), dv.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
+                                     int(bool(causal)), int(window_left), float(scale),
+                                     workspace.data_ptr(), _nbytes(workspace),
+                                     _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_bwd")
     return dq, dk, dv
@@ -288,17 +331,19 @@ def attn_fwd_fp8(q, k, v, q_scale: float, k_scale: float, v_scale: float, causal
     for name, t in (("q", q), ("k", k), ("v", v)):
         if t.dtype != torch.float8_e4m3fn or t.dim() != 4 or not t.is_contiguous() or not t.is_cuda:
             raise ValueError(f"{name} must be a contiguous CUDA float8_e4m3fn [b, s, h, d]")
+    dev = _cuda_device(stream, q=q, k=k, v=v)
     b, s_q, h_q, d = q.shape
     bk, s_k, h_kv, dk = k.shape
     if tuple(v.shape) != tuple(k.shape) or bk != b or dk != d:
         raise ValueError("q, k, v shapes disagree")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
-    rc = load_library().attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                     lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
-                                     int(bool(causal)), float(scale), float(q_scale),
-                                     float(k_scale), float(v_scale), _stream_handle(stream))
+    with _on_device(dev):
+        o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
+        rc = load_library().attn_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                         lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
+                                         int(bool(causal)), float(scale), float(q_scale),
+                                         float(k_scale), float(v_scale), _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_fp8")
     return o, lse
@@ -319,30 +364,20 @@ def attn_fwd_split(q, k, v, causal: bool = False, scale: float | None = None,
     ``n_splits`` None: the library's choice (:func:`num_splits`).  The
     partials go to ``workspace`` (a CUDA uint8 tensor of at least
     :func:`split_workspace_bytes` bytes; allocated here if None)."""
-    import torch
     b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        if not t.is_cuda:
-            raise ValueError(f"{name} must be a CUDA tensor")
+    dev = _cuda_device(stream, q=q, k=k, v=v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    if n_splits is None:
-        n_splits = max(1, num_splits(b, h_q, h_kv, s_q, s_k, causal, d))
-    o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
-    if workspace is None:
-        # Dropped on return while the two kernels may still run: allocated on
-        # their stream, so its memory is not reused before they finish.
-        nbytes = split_workspace_bytes(b, h_q, s_q, n_splits)
-        workspace = _alloc_on(stream, q.device,
-                              lambda: torch.empty(nbytes, dtype=torch.uint8, device=q.device))
-    elif workspace.device != q.device or not workspace.is_contiguous():
-        raise ValueError("workspace must be a contiguous tensor on the inputs' device")
-    rc = load_library().attn_fwd_split(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                       lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
-                                       int(bool(causal)), float(scale), int(n_splits),
-                                       workspace.data_ptr(),
-                                       workspace.numel() * workspace.element_size(),
-                                       _stream_handle(stream))
+    with _on_device(dev):
+        if n_splits is None:
+            n_splits = max(1, num_splits(b, h_q, h_kv, s_q, s_k, causal, d))
+        o, lse = _outputs(q, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
+        workspace = _workspace(q, workspace, split_workspace_bytes(b, h_q, s_q, n_splits), stream)
+        rc = load_library().attn_fwd_split(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                           o.data_ptr(), lse.data_ptr(), b, h_q, h_kv, s_q, s_k,
+                                           d, int(bool(causal)), float(scale), int(n_splits),
+                                           workspace.data_ptr(), _nbytes(workspace),
+                                           _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_split")
     return o, lse
@@ -354,17 +389,16 @@ def attn_fwd_partials(q, k, v, causal: bool = False, scale: float | None = None,
     (normalised over these keys) and LSE_r FP32 [b, h_q, s_q]."""
     import torch
     b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        if not t.is_cuda:
-            raise ValueError(f"{name} must be a CUDA tensor")
+    dev = _cuda_device(stream, q=q, k=k, v=v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
-    o_part, lse_part = _outputs(q, o_part, lse_part, (b, h_q, s_q, d), (b, h_q, s_q), stream,
-                                o_dtype=torch.float32)
-    rc = load_library().attn_fwd_partials(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                          o_part.data_ptr(), lse_part.data_ptr(), b, h_q, h_kv,
-                                          s_q, s_k, d, int(bool(causal)), float(scale),
-                                          _stream_handle(stream))
+    with _on_device(dev):
+        o_part, lse_part = _outputs(q, o_part, lse_part, (b, h_q, s_q, d), (b, h_q, s_q),
+                                    stream, o_dtype=torch.float32)
+        rc = load_library().attn_fwd_partials(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                              o_part.data_ptr(), lse_part.data_ptr(), b, h_q,
+                                              h_kv, s_q, s_k, d, int(bool(causal)),
+                                              float(scale), _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_partials")
     return o_part, lse_part
@@ -385,20 +419,19 @@ def attn_fwd_partials_shard(q, k, v, causal: bool = False, scale: float | None =
     the shard get O_r = 0 and LSE_r = -inf."""
     import torch
     b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
-    for name, t in (("q", q), ("k", k), ("v", v)):
-        if not t.is_cuda:
-            raise ValueError(f"{name} must be a CUDA tensor")
+    dev = _cuda_device(stream, q=q, k=k, v=v)
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     if diag_offset is None:
         diag_offset = s_k - s_q
-    o_part, lse_part = _outputs(q, o_part, lse_part, (b, h_q, s_q, d), (b, h_q, s_q), stream,
-                                o_dtype=torch.float32)
-    rc = load_library().attn_fwd_partials_shard(q.data_ptr(), k.data_ptr(), v.data_ptr(),
-                                                o_part.data_ptr(), lse_part.data_ptr(), b, h_q,
-                                                h_kv, s_q, s_k, d, int(bool(causal)),
-                                                int(diag_offset), float(scale),
-                                                _stream_handle(stream))
+    with _on_device(dev):
+        o_part, lse_part = _outputs(q, o_part, lse_part, (b, h_q, s_q, d), (b, h_q, s_q),
+                                    stream, o_dtype=torch.float32)
+        rc = load_library().attn_fwd_partials_shard(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                                    o_part.data_ptr(), lse_part.data_ptr(), b,
+                                                    h_q, h_kv, s_q, s_k, d, int(bool(causal)),
+                                                    int(diag_offset), float(scale),
+                                                    _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_partials_shard")
     return o_part, lse_part
@@ -417,12 +450,12 @@ def merge_partials(o_parts, lse_parts, o=None, lse=None, stream=None):
     n, b, h_q, s_q, d = o_parts.shape
     if tuple(lse_parts.shape) != (n, b, h_q, s_q):
         raise ValueError("o_parts and lse_parts shapes disagree")
-    if not o_parts.is_cuda or lse_parts.device != o_parts.device:
-        raise ValueError("partials must be CUDA tensors on one device")
-    o, lse = _outputs(o_parts, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
-    rc = load_library().attn_merge_partials(o_parts.data_ptr(), lse_parts.data_ptr(), n, b, h_q,
-                                            s_q, d, o.data_ptr(), lse.data_ptr(),
-                                            _stream_handle(stream))
+    dev = _cuda_device(stream, o_parts=o_parts, lse_parts=lse_parts)
+    with _on_device(dev):
+        o, lse = _outputs(o_parts, o, lse, (b, s_q, h_q, d), (b, h_q, s_q), stream)
+        rc = load_library().attn_merge_partials(o_parts.data_ptr(), lse_parts.data_ptr(), n, b,
+                                                h_q, s_q, d, o.data_ptr(), lse.data_ptr(),
+                                                _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_merge_partials")
     return o, lse
@@ -430,7 +463,8 @@ def merge_partials(o_parts, lse_parts, o=None, lse=None, stream=None):
 
 def attn_fwd_raw(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, b, h_q, h_kv, s_q, s_k, d, causal, scale,
                  stream_handle) -> int:
-    """Direct call of the C entry point; returns its status code."""
+    """Direct call of the C entry point (buffers on the current device);
+    returns its status code."""
     return load_library().attn_fwd(q_ptr, k_ptr, v_ptr, o_ptr, lse_ptr, b, h_q, h_kv, s_q, s_k,
                                    d, int(causal), float(scale), stream_handle)
 
@@ -443,20 +477,26 @@ def attn_fwd_host(q, k, v, o, lse, workspace, causal: bool = False, scale: float
                   stream=None):
     """Forward on HOST tensors (pinned for asynchronous copies) through the
     C entry point that copies in, runs and copies out.  ``workspace`` is a
-    CUDA uint8 tensor of at least :func:`host_workspace_bytes` bytes."""
+    CUDA uint8 tensor of at least :func:`host_workspace_bytes` bytes; the
+    call runs on its device."""
     import torch
     b, s_q, h_q, h_kv, s_k, d = _check_qkv(q, k, v)
+    for name, t in (("q", q), ("k", k), ("v", v)):
+        if t.is_cuda:
+            raise ValueError(f"{name} must be a host tensor (attn_fwd takes device tensors)")
     if scale is None:
         scale = 1.0 / math.sqrt(d)
     _check_out(o, "o", (b, s_q, h_q, d), torch.bfloat16, q.device)
     _check_out(lse, "lse", (b, h_q, s_q), torch.float32, q.device)
-    if not workspace.is_cuda or not workspace.is_contiguous():
+    dev = _cuda_device(stream, workspace=workspace)
+    if not workspace.is_contiguous():
         raise ValueError("workspace must be a contiguous CUDA tensor")
-    rc = load_library().attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
-                                      lse.data_ptr(), b, h_q, h_kv, s_q, s_k, d,
-                                      int(bool(causal)), float(scale), workspace.data_ptr(),
-                                      workspace.numel() * workspace.element_size(),
-                                      _stream_handle(stream))
+    with _on_device(dev):
+        rc = load_library().attn_fwd_host(q.data_ptr(), k.data_ptr(), v.data_ptr(),
+                                          o.data_ptr(), lse.data_ptr(), b, h_q, h_kv, s_q, s_k,
+                                          d, int(bool(causal)), float(scale),
+                                          workspace.data_ptr(), _nbytes(workspace),
+                                          _stream_handle(stream))
     if rc != ATTN_OK:
         raise AttnError(rc, "attn_fwd_host")
     return o, lse
