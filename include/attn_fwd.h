@@ -181,6 +181,14 @@ int attn_fwd_fp8(const void* q, const void* k, const void* v, void* o, float* ls
  * Ordering is that of `stream`: the call starts after the work already
  * queued on it, and it waits for the call's last copy out, so synchronising
  * `stream` covers everything.  Results are bit-identical to attn_fwd's.
+ *
+ * Errors: as attn_fwd, plus ATTN_ERR_INVALID for a null or too small
+ * workspace and ATTN_ERR_ALIGN for a workspace not 256-byte aligned, all
+ * found before anything is queued.  ATTN_ERR_CUDA from a copy or launch that
+ * fails to be queued part way through: o and lse are then unspecified, and
+ * copies of earlier groups may still be running on the library's streams
+ * when the call returns, so synchronise the device (not only `stream`)
+ * before reusing or freeing the buffers.
  */
 int attn_fwd_host(const void* q, const void* k, const void* v, void* o, float* lse,
                   int batch, int h_q, int h_kv, int s_q, int s_k, int d,
