@@ -217,6 +217,23 @@ def whole_job_tflops(world: int, flops_per_step: float, steps: int, max_ms: floa
     return world * flops_per_step * steps / (max_ms * 1e-3) / 1e12
 
 
+def clocks_over_ranks(summary: dict, world: int) -> dict:
+    """The clock record of the whole job from every rank's sampler summary
+    (one small collective after the timed region, taken by every rank): the
+    slowest rank's median SM clock, the reasons seen on any rank, the samples
+    of all ranks and each rank's median."""
+    if world == 1:
+        return summary
+    import torch.distributed as dist
+    every = [None] * world
+    dist.all_gather_object(every, summary)
+    mhz = [s["sm_mhz"] for s in every]
+    known = [m for m in mhz if m is not None]
+    return {"sm_mhz": min(known) if known else None, "sm_max_mhz": every[0]["sm_max_mhz"],
+            "reasons": sorted(set().union(*(s["reasons"] for s in every))),
+            "samples": sum(s["samples"] for s in every), "per_rank_sm_mhz": mhz}
+
+
 # ------------------------------------------------------------------ oracle arm
 def _head_slices(w, q, k, v, i):
     """The i-th (batch, query head) of the workload, cycling through all of
@@ -390,7 +407,7 @@ def run_ours(args, world, rank, local):
         "modes": modes,
         "pct_of_spec_peak": 100.0 * value / world / SPEC_PEAK_TFLOPS,
         "roofline": roofline,
-        "clocks": sampler.summary(),
+        "clocks": clocks_over_ranks(sampler.summary(), world),
         "gpu_launches": 2 * K,
         "kernel_hash": kernel_source_hash(),
         "fwd_kernel_hash": fwd_kernel_hash(),
