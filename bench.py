@@ -669,7 +669,8 @@ def run_e2e(args, w, q, k, v, world):
             attn.attn_fwd_host(qh, kh, vh, oh, lh, ws, causal=causal, scale=w.scale,
                                stream=stream)
 
-    step()
+    for _ in range(max(1, args.warmup)):  # the same warm-up as the device-timed region
+        step()
     torch.cuda.synchronize()
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
