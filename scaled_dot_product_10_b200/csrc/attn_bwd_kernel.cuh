@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::tc_fence_before();
     __syncthreads();
     ptx::tc_fence_after();
-    const uint32_t tmem = *tmem_slot;  // S | dP | dQ at columns 0, 128, 256
+    const uint32_t tmem = *tmem_slot;  // S | dP | dQ | dS at columns 0, 128, 256, 384
     const WaitCtx wc{abort_flag, p.status, p.timeout_ns};
 
     if (warp == kLoadWarp) {
