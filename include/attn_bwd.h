@@ -16,6 +16,9 @@
  *
  * Grouped-query / multi-query attention: dK and dV of key/value head g sum
  * the contributions of every query head of its group (h / (h_q / h_kv) == g).
+ * Keys that no query sees (under a sliding window with s_q < s_k, those
+ * before the first query's window) carry no weight: their dK and dV are
+ * written as zeros.
  *
  * Numerics: S and dP accumulate in FP32 on the tensor cores; P and dS are
  * rounded to BF16 before the products that use them; dQ, dK, dV accumulate

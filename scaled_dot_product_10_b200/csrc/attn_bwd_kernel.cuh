@@ -649,6 +649,31 @@ struct Cursor {
     }
 };
 
+// A key block that no query sees has no item in the main loop (nq = 0):
+// under a sliding window with s_q < s_k the keys before the first query's
+// window are such blocks.  Their dK and dV rows are zero (no weight reaches
+// them); every CTA writes those of the items it would have been dealt.
+__device__ __noinline__ void zero_unseen_key_blocks(const BwdParams& p) {
+    constexpr int kPieces = kHeadDim * 2 / 16;  // 16-byte pieces of one row
+    Cursor c;
+    for (int t = static_cast<int>(blockIdx.x); t < p.num_items;
+         t += static_cast<int>(gridDim.x)) {
+        c.t = t;
+        c.decode(p);
+        if (c.nq > 0) continue;
+        const int r0 = c.kb * kBlockN;
+        const int rows = min(kBlockN, p.s_k - r0);
+        for (int i = static_cast<int>(threadIdx.x); i < rows * kPieces;
+             i += static_cast<int>(blockDim.x)) {
+            const int row = r0 + i / kPieces;
+            const size_t e = ((static_cast<size_t>(c.b) * p.s_k + row) * p.h_kv + c.g) * kHeadDim +
+                             static_cast<size_t>(i % kPieces) * 8;
+            *reinterpret_cast<uint4*>(p.dk + e) = make_uint4(0u, 0u, 0u, 0u);
+            *reinterpret_cast<uint4*>(p.dv + e) = make_uint4(0u, 0u, 0u, 0u);
+        }
+    }
+}
+
 __global__ void __launch_bounds__(kThreads, 1)
     attn_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q,
                          const __grid_constant__ CUtensorMap tm_k,
@@ -666,6 +691,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+    if (p.window_left >= 0) zero_unseen_key_blocks(p);
     if (threadIdx.x == 0) {
         ptx::mbar_init(bar(L::bKFull), 1);
         ptx::mbar_init(bar(L::bKEmpty), 1);

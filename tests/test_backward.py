@@ -115,6 +115,41 @@ def test_bwd_window_zero_gives_zero_dq_dk():
     assert np.max(np.abs(g - dv_ref)) <= MAX_REL * np.max(np.abs(dv_ref))
 
 
+@pytest.mark.parametrize("b,h_q,h_kv,s_q,s_k,w", [
+    (2, 4, 2, 128, 384, 0),     # two whole key blocks before the first window
+    (2, 4, 2, 100, 700, 37),    # unseen keys end inside a block
+    (1, 4, 4, 200, 1000, 130),
+    (8, 8, 4, 128, 1100, 3),    # more key-block items than SMs
+])
+def test_bwd_window_keys_no_query_sees(b, h_q, h_kv, s_q, s_k, w):
+    """Bottom-right window with s_q < s_k: keys before the first query's
+    window (j < s_k - s_q - w) get no weight, so their dK and dV are exactly
+    zero, and whole key blocks of them have no work item of their own.  The
+    outputs start as NaN so that a row nobody wrote shows."""
+    q, k, v, dout = grads_in(b, h_q, h_kv, s_q, s_k, 11460 + s_q + w)
+    qd, kd, vd, dod = q.cuda(), k.cuda(), v.cuda(), dout.cuda()
+    o, lse = attn.attn_fwd_window(qd, kd, vd, w, scale=SCALE)
+    dq, dk, dv = (torch.full_like(t, float("nan")) for t in (qd, kd, vd))
+    attn.attn_bwd(qd, kd, vd, o, lse, dod, causal=True, scale=SCALE, window_left=w, dq=dq,
+                  dk=dk, dv=dv)
+    rc = attn.attn_status()
+    assert rc == attn.ATTN_OK, attn.attn_strerror(rc)
+    unseen = s_k - s_q - w
+    assert torch.all(dk[:, :unseen] == 0) and torch.all(dv[:, :unseen] == 0)
+    ref = oracle.attn_bwd(q, k, v, dout, True, SCALE, window_left=w)
+    for name, g, r in zip(("dQ", "dK", "dV"), (dq, dk, dv), ref):
+        g = g.float().cpu().double().numpy()
+        assert np.all(np.isfinite(g)), f"{name} not finite (a row left unwritten)"
+        if w == 0 and name != "dV":
+            # one visible key per row: dQ = dK = 0 exactly (see above)
+            assert np.max(np.abs(g)) <= 1e-3
+            continue
+        rel = np.linalg.norm(g - r) / max(np.linalg.norm(r), 1e-300)
+        mx = np.max(np.abs(g - r)) / max(np.max(np.abs(r)), 1e-300)
+        assert rel <= REL_L2, f"{name} relative L2 {rel:.3e}"
+        assert mx <= MAX_REL, f"{name} max error {mx:.3e} of max |ref|"
+
+
 @pytest.mark.parametrize("scale", [-0.09, 0.0, 0.5])
 def test_bwd_scales(scale):
     check_bwd(*grads_in(1, 2, 2, 512, 512, 11500), True, scale=scale, what=f"scale={scale}")

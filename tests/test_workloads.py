@@ -36,11 +36,11 @@ def test_headline_workload_counts():
     assert w.input_bytes() == 402_653_184  # above the 126 MB L2: no flush needed
 
 
-@pytest.mark.parametrize("name", sorted(WORKLOADS))
+@pytest.mark.parametrize("name", sorted(n for n, w in WORKLOADS.items() if w.seq <= 4096))
 def test_byte_counts_match_the_tensors(name):
+    """(The formula is the same for the larger workloads; their tensors are
+    not drawn here.)"""
     w = WORKLOADS[name]
-    if w.seq > 4096:
-        pytest.skip("large tensors; the formula is the same")
     q, k, v = workload_qkv(w)
     size = lambda t: t.numel() * t.element_size()  # noqa: E731
     assert w.input_bytes() == size(q) + size(k) + size(v)
