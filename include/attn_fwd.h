@@ -125,7 +125,10 @@ int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float*
  *        launch has work items for max_seqlen_q rows per sequence)
  *   causal, window_left  as attn_fwd / attn_fwd_window (window_left = -1:
  *        none; a window needs causal = 1); causal needs s_q <= s_k per
- *        sequence -- a row that sees no key gets O = 0, LSE = -inf
+ *        sequence.  In a sequence with more query rows than keys the first
+ *        s_q - s_k rows see no key: where such a row shares a 128-row block
+ *        with a row that sees keys it gets O = 0, LSE = -inf, but blocks
+ *        in which no row sees a key are not written at all
  *
  * The host cannot read cu_seqlens: sequences that break the rules above
  * give unspecified values, but every access stays inside the packed
