@@ -503,7 +503,10 @@ def attn_fwd_host(q, k, v, o, lse, workspace, causal: bool = False, scale: float
 
 
 def attn_status(stream=None) -> int:
-    """Synchronise the stream, then read and clear the device status word."""
+    """Synchronise the stream, then read and clear the status word of the
+    current device (the status word is per device: call this with the device
+    of the launches it should cover current, e.g. under
+    ``torch.cuda.device(q.device)``)."""
     return int(load_library().attn_status(_stream_handle(stream)))
 
 
