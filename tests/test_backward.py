@@ -96,6 +96,13 @@ def test_bwd_rectangular(s_q, s_k, causal):
               what=f"{s_q}x{s_k} causal={causal}")
 
 
+@pytest.mark.parametrize("s_q,s_k", [(700, 300), (1000, 129)])
+def test_bwd_more_queries_than_keys(s_q, s_k):
+    # Without a mask s_q > s_k is allowed: more query blocks than key blocks,
+    # a ragged last key block (keys past s_k get no weight in dQ).
+    check_bwd(*grads_in(2, 4, 2, s_q, s_k, 11350 + s_q), False, what=f"{s_q}x{s_k}")
+
+
 @pytest.mark.parametrize("w", [1, 100, 255])
 def test_bwd_window(w):
     check_bwd(*grads_in(1, 4, 4, 1000, 1000, 11400 + w), True, window_left=w, what=f"w={w}")
