@@ -652,7 +652,9 @@ struct Cursor {
 // A key block that no query sees has no item in the main loop (nq = 0):
 // under a sliding window with s_q < s_k the keys before the first query's
 // window are such blocks.  Their dK and dV rows are zero (no weight reaches
-// them); every CTA writes those of the items it would have been dealt.
+// them).  The CTAs share the items by a grid stride (each item t is
+// visited by CTA t mod gridDim.x alone) and write the rows of those with
+// nq = 0; the main loop never touches these rows.
 __device__ __noinline__ void zero_unseen_key_blocks(const BwdParams& p) {
     constexpr int kPieces = kHeadDim * 2 / 16;  // 16-byte pieces of one row
     Cursor c;
