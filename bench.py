@@ -696,6 +696,10 @@ def main():
         rank = int(os.environ.get("RANK", "0"))
         return run_reference(args, world, rank)
     world, rank, local = dist_setup(args)
+    if args.gpus != world and rank == 0:
+        # The line reports the ranks that actually ran (n_gpus = WORLD_SIZE).
+        print(f"bench.py: --gpus {args.gpus} but {world} rank(s) running; launch N > 1 with "
+              "torchrun --nproc-per-node N", file=sys.stderr, flush=True)
     if args.only:
         from scaled_dot_product_10_b200 import attn
         attn.load_library()
